@@ -1,0 +1,502 @@
+#!/usr/bin/env python
+"""Benchmark of the SATA attention hot path (prefill + decode, d_K = d_V = 64, P = 4).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0.  ``value`` is prefill throughput in tokens/s summed
+over all ranks on the long bf16 prefill (B=1, H=8, N=16384): one step is one
+``sata_prefill`` call (basis tables, feature expansion, chunk states, readout,
+normalisation, final state).  The ``decode`` object reports the batched
+decode workload (B=32, H=8, state of an N=8192 bf16 prefill): one step is one
+``sata_decode_step`` call for all 32 sequences.  Inputs are seeded synthetic
+N(0,1) (``sata_inputs``).  Timing: CUDA events on the launching stream; prefill
+steps are separated by an L2 flush (a 256 MiB write) outside the events; the
+decode state (3.19 GB) is larger than L2.  Multi-GPU runs are weak scaling:
+every rank processes its own independent batch of heads, no collective on the
+data path; times are the max over ranks.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (a
+bounded sample of the same workloads, reported in the same unit).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "tokens/sec/GPU (prefill & decode) at d_K=64,P=4; % tensor / HBM roofline"
+PREFILL = dict(B=1, H=8, N=16384, dK=64, dV=64, P=4)
+DECODE = dict(B=32, H=8, N=8192, dK=64, dV=64, P=4)
+WORKLOAD = ("prefill B=1,H=8,N=16384,dK=dV=64,P=4 bf16 (one sata_prefill per step); "
+            "decode B=32,H=8,dK=dV=64,P=4 fp32 state of an N=8192 bf16 prefill "
+            "(one sata_decode_step per step)")
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]),
+                "sm_max_mhz": float(p.get("sm_max_mhz", 1965.0)), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def basis_m(dK, P):
+    return math.comb(dK + P - 1, P - 1)
+
+
+# --------------------------------------------------------------- clocks sampler
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        mhz, mx, reasons = [], [], set()
+        for r in self.rows:
+            try:
+                mhz.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [x for x in mhz if x > 0.5 * max(mhz)] or mhz
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# --------------------------------------------------------------- traffic record
+def traffic_record(kernel: str):
+    """Per-launch DRAM bytes of ``kernel`` from the committed ncu summary, or
+    None when the kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    r = rec.get(kernel)
+    if not r or r.get("source_sha") != source_sha():
+        return None
+    return r.get("bytes_per_launch")
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_cost_attention_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+# --------------------------------------------------------------- oracle timing
+def oracle_prefill_sample(rows: int, seed: int = 0):
+    """fp64 oracle on a bounded sample of the prefill workload: `rows` query rows
+    (evenly spaced over N) of one head through the quadratic form, and the state
+    accumulation over `rows` tokens.  Returns (seconds, equivalent tokens)."""
+    import numpy as np
+
+    import oracle
+    from sata_inputs import make_qkv
+
+    w = PREFILL
+    q, k, v = make_qkv(1, 1, w["N"], w["dK"], w["dV"], seed=seed, dtype="bf16")
+    qq, kk, vv = (t.double().numpy()[0, 0] for t in (q, k, v))
+    idx = np.linspace(0, w["N"] - 1, rows).astype(np.int64)
+    t0 = time.perf_counter()
+    scale = 1.0 / math.sqrt(w["dK"])
+    for i0 in range(0, rows, 256):
+        ii = idx[i0:i0 + 256]
+        s = (qq[ii] @ kk.T) * scale
+        t = oracle.taylor_kernel(s, w["P"])
+        t = np.where(np.arange(w["N"])[None, :] <= ii[:, None], t, 0.0)
+        _ = t @ vv, t.sum(axis=1)
+    oracle.final_state(k[:, :, :rows], v[:, :, :rows], w["P"])
+    dt = time.perf_counter() - t0
+    # one head of H: `rows` token rows count as rows/H tokens of the whole batch
+    return dt, rows / w["H"]
+
+
+def oracle_decode_sample(heads: int, seed: int = 1):
+    """fp64 oracle decode step on `heads` heads from a random state.  Returns
+    (seconds, equivalent tokens of the B=32,H=8 step)."""
+    import numpy as np
+
+    import oracle
+
+    w = DECODE
+    r = np.random.default_rng(seed)
+    m = basis_m(w["dK"], w["P"])
+    S = r.standard_normal((1, heads, m, w["dV"] + 1))
+    qv = r.standard_normal((1, heads, w["dK"]))
+    kv = r.standard_normal((1, heads, w["dK"]))
+    vv = r.standard_normal((1, heads, w["dV"]))
+    t0 = time.perf_counter()
+    oracle.decode_step(qv, kv, vv, S, w["P"])
+    dt = time.perf_counter() - t0
+    return dt, heads / w["H"]
+
+
+def host_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        info = threadpool_info()
+        return max(int(i.get("num_threads", 1)) for i in info) if info else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(budget_s: float = 20.0):
+    rows = 2048
+    dt, tok = oracle_prefill_sample(rows)
+    while dt < budget_s * 0.4 and rows < PREFILL["N"]:
+        rows = min(PREFILL["N"], rows * 2)
+        dt, tok = oracle_prefill_sample(rows)
+    ddt, dtok = oracle_decode_sample(2)
+    return {"value": tok / dt, "unit": "tokens/s", "cores": host_threads(), "kind": "oracle",
+            "sample": f"prefill: {rows} query rows evenly spaced over N=16384 of 1 of 8 heads "
+                      f"(quadratic form) + state over {rows} tokens, fp64 numpy, {dt:.1f} s",
+            "decode": {"value": dtok / ddt, "unit": "tokens/s",
+                       "sample": f"1 decode step of 2 of the 256 heads from a random state, "
+                                 f"{ddt:.2f} s"}}
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import linear_cost_attention_b200 as sata
+    from sata_inputs import DecodeStream, make_qkv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pk = peaks()
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        import torch.distributed as dist
+
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    phys = vis[local_rank] if local_rank < len(vis) else str(local_rank)
+    sampler = ClockSampler(int(phys) if phys.strip().isdigit() else local_rank)
+
+    # ---------------- prefill
+    w = PREFILL
+    m = basis_m(w["dK"], w["P"])
+    q, k, v = make_qkv(w["B"], w["H"], w["N"], w["dK"], w["dV"], seed=20261204 + 1000 * rank,
+                       dtype="bf16")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    out = torch.empty(w["B"], w["H"], w["N"], w["dV"], device=dev)
+    state = torch.empty(w["B"], w["H"], m, w["dV"] + 1, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def prefill():
+        sata.sata_prefill(qd, kd, vd, out, state, w["B"], w["H"], w["N"], w["dK"], w["dV"],
+                          w["P"], torch.bfloat16, stream)
+
+    for _ in range(args.warmup):
+        prefill()
+    torch.cuda.synchronize()
+    sata.sata_profile_enable(True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    kern = {}
+    launches = 0
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        prefill()
+        ev[i][1].record(stream)
+        prof = sata.sata_profile_read()  # syncs on this step's kernel events
+        launches += len(prof)
+        for name, ms in prof:
+            kern.setdefault(name, []).append(ms)
+    torch.cuda.synchronize()
+    barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(step_ms))
+    prefill_tokens = w["B"] * w["N"]
+    value = world * args.steps * prefill_tokens / (total_ms / 1e3)
+    assert sata.sata_get_error() == sata.SATA_OK
+
+    # dominant kernel of the prefill step
+    share = {n: sum(x) for n, x in kern.items()}
+    top = max(share, key=share.get)
+    top_ms = statistics.mean(kern[top])
+    per_tok_head = 2 * (w["dV"] + 1) * m  # one of the two state contractions
+    if top in ("tc_readout", "tc_chunk_states", "simt_readout", "simt_chunk_states"):
+        alg = w["B"] * w["H"] * w["N"] * per_tok_head
+    else:
+        alg = w["B"] * w["H"] * w["N"] * 2 * per_tok_head
+    if top.startswith("tc_"):
+        bound, peak, unit = "tensor", pk["bf16_tflops"], "TFLOP/s"
+    else:
+        # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
+        bound, peak, unit = "alu", 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12, "TFLOP/s"
+    achieved = alg / (top_ms / 1e3) / 1e12
+    roof = {"bound": bound, "kernel": top, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": traffic_record(top),
+            "peak_source": pk["source"] if bound == "tensor" else "derived: 148x128x2 flop x sm_max_mhz",
+            "kernel_ms": top_ms, "algorithmic_flop_per_launch": alg,
+            "kernel_share": {n: s / sum(share.values()) for n, s in share.items()}}
+
+    # e2e prefill: pinned host inputs, H2D + call + D2H of out and state per step
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    st_h = torch.empty(state.shape, dtype=state.dtype, pin_memory=True)
+    e2e_ms = []
+    sata.sata_profile_enable(False)
+    for i in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        prefill()
+        out_h.copy_(out, non_blocking=True)
+        st_h.copy_(state, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_total = max_over_ranks(sum(e2e_ms))
+    e2e = {"value": world * args.steps * prefill_tokens / (e2e_total / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (q, k, v)),
+           "d2h_bytes_per_step": out.numel() * 4 + state.numel() * 4}
+    del qd, kd, vd, out, state, q, k, v, qh, kh, vh, out_h, st_h
+
+    # ---------------- decode
+    dw = DECODE
+    dm = basis_m(dw["dK"], dw["P"])
+    q, k, v = make_qkv(dw["B"], dw["H"], dw["N"], dw["dK"], dw["dV"],
+                       seed=20261205 + 100 + 1000 * rank, dtype="bf16")
+    dstate = torch.empty(dw["B"], dw["H"], dm, dw["dV"] + 1, device=dev)
+    dout = torch.empty(dw["B"], dw["H"], w["dV"], device=dev)
+    sata.sata_prefill(q.to(dev), k.to(dev), v.to(dev), torch.empty(dw["B"], dw["H"], dw["N"], dw["dV"], device=dev),
+                      dstate, dw["B"], dw["H"], dw["N"], dw["dK"], dw["dV"], dw["P"],
+                      torch.bfloat16, stream)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    ds = DecodeStream(5)
+    nsteps = args.decode_steps
+    toks = [tuple(t.to(dev) for t in ds.next()) for _ in range(args.warmup + nsteps)]
+    for i in range(args.warmup):
+        qt, kt, vt = toks[i]
+        sata.sata_decode_step(qt, kt, vt, dstate, dout, dw["B"], dw["H"], dw["dK"], dw["dV"],
+                              dw["P"], torch.bfloat16, stream)
+    torch.cuda.synchronize()
+    sata.sata_profile_enable(True)
+    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(nsteps)]
+    dk = {}
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(nsteps):
+        qt, kt, vt = toks[args.warmup + i]
+        dev_ev[i][0].record(stream)
+        sata.sata_decode_step(qt, kt, vt, dstate, dout, dw["B"], dw["H"], dw["dK"], dw["dV"],
+                              dw["P"], torch.bfloat16, stream)
+        dev_ev[i][1].record(stream)
+        for name, ms in sata.sata_profile_read():
+            dk.setdefault(name, []).append(ms)
+            launches += 1
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    sata.sata_profile_enable(False)
+    dms = [a.elapsed_time(b) for a, b in dev_ev]
+    dtotal = max_over_ranks(sum(dms))
+    dvalue = world * nsteps * dw["B"] / (dtotal / 1e3)
+    dbytes = 2 * dw["B"] * dw["H"] * dm * (dw["dV"] + 1) * 4
+    dkern_ms = statistics.mean(dk["decode_stream"])
+    dach = dbytes / (dkern_ms / 1e3) / 1e9
+    q4 = max(1, nsteps // 4)
+    decode = {
+        "value": dvalue, "unit": "tokens/s", "ms_per_step": dtotal / nsteps,
+        "steps": nsteps, "context_start": dw["N"] + args.warmup,
+        "latency_ms_first_quarter_median": statistics.median(dms[:q4]),
+        "latency_ms_last_quarter_median": statistics.median(dms[-q4:]),
+        "roofline": {"bound": "hbm", "kernel": "decode_stream", "achieved": dach,
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dach / pk["hbm_gbs"],
+                     "traffic": traffic_record("decode_stream"),
+                     "peak_source": pk["source"], "kernel_ms": dkern_ms,
+                     "algorithmic_bytes_per_launch": dbytes},
+    }
+    # e2e decode: H2D of the step's q,k,v from pinned host, D2H of out
+    hq = [tuple(t.pin_memory() for t in ds.next()) for _ in range(min(nsteps, 64))]
+    dout_h = torch.empty(dout.shape, pin_memory=True)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    qt, kt, vt = toks[0]
+    a.record(stream)
+    for qh_, kh_, vh_ in hq:
+        qt.copy_(qh_, non_blocking=True)
+        kt.copy_(kh_, non_blocking=True)
+        vt.copy_(vh_, non_blocking=True)
+        sata.sata_decode_step(qt, kt, vt, dstate, dout, dw["B"], dw["H"], dw["dK"], dw["dV"],
+                              dw["P"], torch.bfloat16, stream)
+        dout_h.copy_(dout, non_blocking=True)
+    b.record(stream)
+    b.synchronize()
+    de2e = max_over_ranks(a.elapsed_time(b))
+    decode["e2e"] = {"value": world * len(hq) * dw["B"] / (de2e / 1e3), "unit": "tokens/s",
+                     "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hq[0]),
+                     "d2h_bytes_per_step": dout.numel() * 4}
+    assert sata.sata_get_error() == sata.SATA_OK
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded i.i.d. N(0,1) q,k,v cast to bf16",
+        "config": {"workload": WORKLOAD, "global_batch": world * PREFILL["B"] * PREFILL["H"],
+                   "seq_len": PREFILL["N"], "parallelism": f"dp{world} (independent heads)",
+                   "l2": "prefill: 256 MiB L2 flush between timed steps; decode: 3.19 GB state > L2",
+                   "decode_steps": nsteps},
+        "roofline": roof, "decode": decode, "e2e": e2e, "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    return line
+
+
+# --------------------------------------------------------------- reference arm
+def run_reference(args):
+    per_step = []
+    rows = args.ref_rows
+    for i in range(args.warmup + args.steps):
+        dt, tok = oracle_prefill_sample(rows, seed=i)
+        if i >= args.warmup:
+            per_step.append((dt, tok))
+    t = sum(d for d, _ in per_step)
+    tok = sum(x for _, x in per_step)
+    ddt, dtok = oracle_decode_sample(2)
+    value = tok / t
+    sample = (f"each step: {rows} query rows evenly spaced over N=16384 of 1 of 8 heads "
+              f"(quadratic form) + state over {rows} tokens; fp64 numpy on host cores")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: seeded i.i.d. N(0,1) q,k,v cast to bf16",
+        "config": {"workload": WORKLOAD, "global_batch": PREFILL["B"] * PREFILL["H"],
+                   "seq_len": PREFILL["N"], "parallelism": "host threads"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_threads(),
+                         "kind": "oracle", "sample": sample},
+        "decode": {"value": dtok / ddt, "unit": "tokens/s",
+                   "sample": "1 decode step of 2 of 256 heads from a random state"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=128)
+    ap.add_argument("--ref-rows", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    line = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,137 @@
+/*
+ * sata.h — C ABI of the B200 (sm_100a) library for causal SATA attention
+ * (symmetry-aware Taylor approximation).
+ *
+ * Operation.  Per head, with s_ij = q_i . k_j / sqrt(dK) and
+ * T_P(s) = sum_{p=0}^{P-1} s^p / p!  (exp truncated to degrees 0..P-1):
+ *     out_i = sum_{j<=i} T_P(s_ij) v_j  /  sum_{j<=i} T_P(s_ij)
+ * evaluated through the feature map over the minimal basis of each order-p
+ * symmetric tensor (index tuples i_1 <= ... <= i_p, the tables M_p) and a
+ * fixed-size state S of shape [m, dV+1], m = C(dK+P-1, P-1), whose last column
+ * is the normaliser.
+ *   Source: "对称性感知泰勒近似注意力机制的恒定计算成本工程实现" (blog.hotdry.top),
+ *   sections "对称张量分解的核心洞察" (Taylor expansion, minimal basis
+ *   C(dK+p-1,p), fixed index tables M_p) and "恒定计算成本的工程实现"
+ *   (state of (dV+1) x C(dK+P-1,P-1) elements, per-token update and readout).
+ *   Layout (batch, heads, seq, dim) and the dim**-0.5 scale follow
+ *   "Transformer 注意力机制变体与长序列建模优化" (mokono.cn), section 2.1.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are CUDA device (or managed) memory of the current
+ *     device, owned by the caller; the library never frees or retains them.
+ *     Every base pointer must be 16-byte aligned.
+ *   - Row-major contiguous layouts:
+ *       q, k   [B, H, N, dK]     dtype = SATA_F32 (float) or SATA_BF16 (bfloat16)
+ *       v      [B, H, N, dV]     same dtype as q, k
+ *       out    [B, H, N, dV]     float
+ *       state  [B, H, m, dV+1]   float; row r is basis row r in degree-major,
+ *                                lexicographic order (the order of
+ *                                sata_index_table); column dV is the normaliser
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous; no call synchronises the device except
+ *     sata_get_error.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call returns a status and launches nothing.  Nothing throws
+ *     across this interface.
+ *   - Supported: dK, dV in {8, 16, 32, 64}; 1 <= P <= 4; B, H, N >= 1 with
+ *     B*H*N*max(dK,dV) < 2^31.
+ *   - The library lazily allocates, per device, its basis tables and a
+ *     grow-only scratch workspace (cudaMalloc); both live until sata_release()
+ *     or process exit.  Calls from several host threads are serialised by an
+ *     internal mutex.
+ */
+#ifndef SATA_H_
+#define SATA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *sata_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  SATA_OK = 0,
+  SATA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, aliasing   */
+  SATA_ERR_UNSUPPORTED = 2, /* dK, dV or P outside the supported set        */
+  SATA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed          */
+  SATA_ERR_NOMEM = 4,       /* workspace allocation failed                   */
+  SATA_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up            */
+} sata_status;
+
+typedef enum { SATA_F32 = 0, SATA_BF16 = 1 } sata_dtype;
+
+/* Number of basis rows m = sum_{p<P} C(dK+p-1, p) = C(dK+P-1, P-1)
+ * ("恒定计算成本的工程实现": state size (dV+1) x C(dK+P-1, P-1)).
+ * Host only.  Returns -1 if dK < 1 or P < 1 or the result overflows int64. */
+int64_t sata_basis_size(int dK, int P);
+
+/* Writes M_p ("对称张量分解的核心洞察": index tuples of the upper-triangular
+ * region), i.e. every tuple 0 <= i_1 <= ... <= i_p < dK in lexicographic
+ * order, row-major [C(dK+p-1,p), p] int32, into host_out.  Host only.
+ * cap_elems is the capacity of host_out in int32 elements.  Returns the number
+ * of rows (>= 1; p = 0 has one empty row and writes nothing), or -1 on a bad
+ * argument (dK < 1, p < 0, host_out NULL while p > 0) or when cap_elems is too
+ * small (nothing is written then). */
+int64_t sata_index_table(int dK, int p, int32_t *host_out, int64_t cap_elems);
+
+/* Causal prefill from a zero state.  Writes out (every token) and overwrites
+ * state with S after the last token.  q, k, v, out, state: see layouts above;
+ * out and state must not overlap each other or the inputs.
+ * The bf16 path computes the feature products in fp32, rounds features, the
+ * chunk-boundary states and the in-chunk Taylor scores to bf16 for the tensor
+ * cores, and accumulates in fp32; the fp32 path stays in fp32 throughout.
+ * Returns SATA_OK, SATA_ERR_INVALID_ARG, SATA_ERR_UNSUPPORTED, SATA_ERR_NOMEM
+ * or SATA_ERR_CUDA. */
+int sata_prefill(const void *q, const void *k, const void *v, float *out,
+                 float *state, int B, int H, int N, int dK, int dV, int P,
+                 sata_dtype dt, sata_stream_t stream);
+
+/* One single-token step for each of B*H heads ("恒定计算成本的工程实现":
+ * per-token procedure at constant cost): state += phi(k) [v, 1]^T in place,
+ * then out = (phi(q)^T state)[:dV] / (phi(q)^T state)[dV].  The token attends
+ * to itself and to everything folded into state.
+ * q, k [B, H, dK]; v [B, H, dV] (dtype dt); state [B, H, m, dV+1] float,
+ * updated in place; out [B, H, dV] float.
+ * Returns SATA_OK, SATA_ERR_INVALID_ARG, SATA_ERR_UNSUPPORTED, SATA_ERR_NOMEM
+ * or SATA_ERR_CUDA. */
+int sata_decode_step(const void *q, const void *k, const void *v, float *state,
+                     float *out, int B, int H, int dK, int dV, int P,
+                     sata_dtype dt, sata_stream_t stream);
+
+/* Synchronises `stream`, then reports (and clears) the first device-side error
+ * recorded by this library's kernels on the current device (a bounded wait
+ * that gave up -> SATA_ERR_TIMEOUT) or a pending CUDA error (-> SATA_ERR_CUDA).
+ * Returns SATA_OK when there is none. */
+int sata_get_error(sata_stream_t stream);
+
+/* Static string for a status code (never NULL). Host only. */
+const char *sata_status_string(int status);
+
+/* Measurement hook (no counterpart on the pages; used by the benchmark).
+ * sata_profile_enable(1) makes every later prefill/decode call record a pair
+ * of CUDA events on its stream around each kernel it launches;
+ * sata_profile_enable(0) stops it (the default).  Returns the previous
+ * setting.  Host only. */
+int sata_profile_enable(int on);
+
+/* Synchronises on the events of the most recent profiled call and writes, for
+ * each kernel that call launched (in launch order, at most cap), its duration
+ * in milliseconds to ms_out[i] and its kernel id to ids_out[i] (either pointer
+ * may be NULL).  Returns the number of kernels the call launched (may exceed
+ * cap), or -1 on a CUDA error. */
+int sata_profile_read(float *ms_out, int *ids_out, int cap);
+
+/* Static name of a kernel id reported by sata_profile_read (never NULL). */
+const char *sata_kernel_name(int id);
+
+/* Frees the library's device tables and workspace on every device it touched.
+ * The caller must make sure no library work is still in flight. */
+void sata_release(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SATA_H_ */

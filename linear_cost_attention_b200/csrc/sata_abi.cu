@@ -1,0 +1,298 @@
+// C ABI of the SATA attention library: argument validation, per-device caches
+// (basis tables, scratch workspace, device error word) and kernel dispatch.
+// Declarations and the contract of every entry point are in include/sata.h.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "sata_internal.h"
+
+namespace sata {
+namespace {
+
+struct DeviceCache {
+  std::map<std::pair<int, int>, DeviceBasis *> bases;
+  std::map<cudaStream_t, std::pair<void *, size_t>> workspaces;
+  int *err = nullptr;  // device error word
+};
+
+std::mutex g_mutex;
+std::map<int, DeviceCache> g_devices;
+
+DeviceCache &cache_for_current_device(int *dev_out) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev_out) *dev_out = dev;
+  return g_devices[dev];
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  const uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+bool supported_dim(int d) { return d == 8 || d == 16 || d == 32 || d == 64; }
+
+void free_basis(DeviceBasis *b) {
+  if (!b) return;
+  cudaFree(b->idx);
+  cudaFree(b->w);
+  cudaFree(b->tile_desc);
+  cudaFree(b->tile_row);
+  delete b;
+}
+
+}  // namespace
+
+const DeviceBasis *get_device_basis(int dK, int P, int *status) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCache &dc = cache_for_current_device(nullptr);
+  auto it = dc.bases.find({dK, P});
+  if (it != dc.bases.end()) return it->second;
+  HostBasis hb = build_host_basis(dK, P);
+  std::vector<uint32_t> idx(hb.m);
+  std::vector<float> w(hb.m);
+  for (int64_t r = 0; r < hb.m; ++r) {
+    idx[r] = (uint32_t)hb.ix[3 * r] | (uint32_t)hb.ix[3 * r + 1] << 8 |
+             (uint32_t)hb.ix[3 * r + 2] << 16 | (uint32_t)hb.degree[r] << 24;
+    w[r] = (float)hb.weight[r];
+  }
+  DeviceBasis *db = new DeviceBasis();
+  db->dK = dK;
+  db->P = P;
+  db->m = hb.m;
+  bool ok = cudaMalloc(&db->idx, hb.m * sizeof(uint32_t)) == cudaSuccess &&
+            cudaMalloc(&db->w, hb.m * sizeof(float)) == cudaSuccess &&
+            cudaMemcpy(db->idx, idx.data(), hb.m * sizeof(uint32_t), cudaMemcpyHostToDevice) ==
+                cudaSuccess &&
+            cudaMemcpy(db->w, w.data(), hb.m * sizeof(float), cudaMemcpyHostToDevice) ==
+                cudaSuccess;
+  if (!ok) {
+    free_basis(db);
+    *status = SATA_ERR_NOMEM;
+    return nullptr;
+  }
+  dc.bases[{dK, P}] = db;
+  return db;
+}
+
+void *get_workspace(cudaStream_t stream, size_t bytes, int *status) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCache &dc = cache_for_current_device(nullptr);
+  auto &ws = dc.workspaces[stream];
+  if (ws.second >= bytes && ws.first) return ws.first;
+  if (ws.first) {
+    // the previous buffer may still be read by work queued on this stream
+    cudaStreamSynchronize(stream);
+    cudaFree(ws.first);
+    ws.first = nullptr;
+    ws.second = 0;
+  }
+  size_t sz = bytes + (bytes >> 3);  // some headroom for growth
+  sz = (sz + 255) & ~(size_t)255;
+  if (cudaMalloc(&ws.first, sz) != cudaSuccess) {
+    cudaGetLastError();
+    ws.first = nullptr;
+    *status = SATA_ERR_NOMEM;
+    return nullptr;
+  }
+  ws.second = sz;
+  return ws.first;
+}
+
+int *device_error_ptr() {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCache &dc = cache_for_current_device(nullptr);
+  if (!dc.err) {
+    if (cudaMalloc(&dc.err, sizeof(int)) != cudaSuccess) {
+      cudaGetLastError();
+      dc.err = nullptr;
+      return nullptr;
+    }
+    cudaMemset(dc.err, 0, sizeof(int));
+  }
+  return dc.err;
+}
+
+int read_and_clear_device_error() {
+  int *p = device_error_ptr();
+  if (!p) return 0;
+  int h = 0;
+  if (cudaMemcpy(&h, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return -1;
+  if (h) cudaMemset(p, 0, sizeof(int));
+  return h;
+}
+
+// ---------------------------------------------------------------- profiling
+namespace {
+struct ProfRec {
+  int id;
+  cudaEvent_t a, b;
+};
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;       // records of the most recent call
+std::vector<cudaEvent_t> g_events;  // pool, reused
+size_t g_next_event = 0;
+
+cudaEvent_t prof_event() {
+  if (g_next_event == g_events.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    g_events.push_back(e);
+  }
+  return g_events[g_next_event++];
+}
+}  // namespace
+
+void prof_call_begin() {
+  if (!g_prof_on) return;
+  g_prof.clear();
+  g_next_event = 0;
+}
+
+void prof_kernel_begin(cudaStream_t s, int id) {
+  if (!g_prof_on) return;
+  ProfRec r{id, prof_event(), prof_event()};
+  if (r.a) cudaEventRecord(r.a, s);
+  g_prof.push_back(r);
+}
+
+void prof_kernel_end(cudaStream_t s) {
+  if (!g_prof_on || g_prof.empty()) return;
+  if (g_prof.back().b) cudaEventRecord(g_prof.back().b, s);
+}
+
+}  // namespace sata
+
+using namespace sata;
+
+extern "C" int sata_profile_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  const int prev = g_prof_on ? 1 : 0;
+  g_prof_on = on != 0;
+  return prev;
+}
+
+extern "C" int sata_profile_read(float *ms_out, int *ids_out, int cap) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  const int n = (int)g_prof.size();
+  for (int i = 0; i < n && i < cap; ++i) {
+    float ms = 0.f;
+    if (!g_prof[i].a || !g_prof[i].b) return -1;
+    if (cudaEventSynchronize(g_prof[i].b) != cudaSuccess) return -1;
+    if (cudaEventElapsedTime(&ms, g_prof[i].a, g_prof[i].b) != cudaSuccess) return -1;
+    if (ms_out) ms_out[i] = ms;
+    if (ids_out) ids_out[i] = g_prof[i].id;
+  }
+  return n;
+}
+
+extern "C" const char *sata_kernel_name(int id) {
+  switch (id) {
+    case K_SIMT_CHUNK_STATES: return "simt_chunk_states";
+    case K_SIMT_READOUT: return "simt_readout";
+    case K_DECODE_STREAM: return "decode_stream";
+    case K_DECODE_FINALIZE: return "decode_finalize";
+    case K_TC_CHUNK_STATES: return "tc_chunk_states";
+    case K_TC_READOUT: return "tc_readout";
+    case K_TC_PREP: return "tc_prep";
+  }
+  return "unknown";
+}
+
+extern "C" int sata_prefill(const void *q, const void *k, const void *v, float *out,
+                            float *state, int B, int H, int N, int dK, int dV, int P,
+                            sata_dtype dt, sata_stream_t stream) {
+  if (!q || !k || !v || !out || !state) return SATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state))
+    return SATA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return SATA_ERR_INVALID_ARG;
+  if (dt != SATA_F32 && dt != SATA_BF16) return SATA_ERR_INVALID_ARG;
+  if (!supported_dim(dK) || !supported_dim(dV) || P < 1 || P > 4) return SATA_ERR_UNSUPPORTED;
+  const long long BHN = (long long)B * H * N;
+  if (BHN * (dK > dV ? dK : dV) >= (1LL << 31)) return SATA_ERR_INVALID_ARG;
+  const int64_t m = count_basis(dK, P);
+  const size_t es = dt == SATA_F32 ? 4 : 2;
+  const size_t nq = BHN * dK * es, nv = BHN * dV * es, no = BHN * dV * 4;
+  const size_t ns = (size_t)B * H * m * (dV + 1) * 4;
+  if (overlaps(out, no, q, nq) || overlaps(out, no, k, nq) || overlaps(out, no, v, nv) ||
+      overlaps(state, ns, q, nq) || overlaps(state, ns, k, nq) || overlaps(state, ns, v, nv) ||
+      overlaps(out, no, state, ns))
+    return SATA_ERR_INVALID_ARG;
+  int st = SATA_OK;
+  const DeviceBasis *basis = get_device_basis(dK, P, &st);
+  if (!basis) return st;
+  prof_call_begin();
+  return launch_prefill_simt(q, k, v, out, state, B, H, N, dK, dV, P, dt == SATA_BF16, basis,
+                             (cudaStream_t)stream);
+}
+
+extern "C" int sata_decode_step(const void *q, const void *k, const void *v, float *state,
+                                float *out, int B, int H, int dK, int dV, int P, sata_dtype dt,
+                                sata_stream_t stream) {
+  if (!q || !k || !v || !out || !state) return SATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state))
+    return SATA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1) return SATA_ERR_INVALID_ARG;
+  if (dt != SATA_F32 && dt != SATA_BF16) return SATA_ERR_INVALID_ARG;
+  if (!supported_dim(dK) || !supported_dim(dV) || P < 1 || P > 4) return SATA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  const int64_t m = count_basis(dK, P);
+  if (BH * m * (dV + 1) >= (1LL << 40)) return SATA_ERR_INVALID_ARG;
+  const size_t es = dt == SATA_F32 ? 4 : 2;
+  const size_t nq = BH * dK * es, nv = BH * dV * es, no = BH * dV * 4;
+  const size_t ns = (size_t)BH * m * (dV + 1) * 4;
+  if (overlaps(out, no, q, nq) || overlaps(out, no, k, nq) || overlaps(out, no, v, nv) ||
+      overlaps(state, ns, q, nq) || overlaps(state, ns, k, nq) || overlaps(state, ns, v, nv) ||
+      overlaps(out, no, state, ns))
+    return SATA_ERR_INVALID_ARG;
+  int st = SATA_OK;
+  const DeviceBasis *basis = get_device_basis(dK, P, &st);
+  if (!basis) return st;
+  prof_call_begin();
+  return launch_decode(q, k, v, state, out, B, H, dK, dV, P, dt == SATA_BF16, basis,
+                       (cudaStream_t)stream);
+}
+
+extern "C" int sata_get_error(sata_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return SATA_ERR_CUDA;
+  }
+  if (cudaGetLastError() != cudaSuccess) return SATA_ERR_CUDA;
+  const int code = read_and_clear_device_error();
+  if (code < 0) return SATA_ERR_CUDA;
+  return code == 0 ? SATA_OK : SATA_ERR_TIMEOUT;
+}
+
+extern "C" const char *sata_status_string(int status) {
+  switch (status) {
+    case SATA_OK: return "SATA_OK";
+    case SATA_ERR_INVALID_ARG: return "SATA_ERR_INVALID_ARG: invalid argument";
+    case SATA_ERR_UNSUPPORTED: return "SATA_ERR_UNSUPPORTED: dK, dV or P not supported";
+    case SATA_ERR_CUDA: return "SATA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case SATA_ERR_NOMEM: return "SATA_ERR_NOMEM: device allocation failed";
+    case SATA_ERR_TIMEOUT: return "SATA_ERR_TIMEOUT: a device-side wait gave up";
+  }
+  return "unknown sata status";
+}
+
+extern "C" void sata_release(void) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto &kv : g_devices) {
+    cudaSetDevice(kv.first);
+    for (auto &b : kv.second.bases) free_basis(b.second);
+    for (auto &w : kv.second.workspaces) cudaFree(w.second.first);
+    cudaFree(kv.second.err);
+  }
+  g_devices.clear();
+  cudaSetDevice(cur);
+}

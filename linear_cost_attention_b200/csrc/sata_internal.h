@@ -1,0 +1,80 @@
+// Internal declarations shared by the library's translation units.
+// Not part of the public ABI (see include/sata.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/sata.h"
+
+namespace sata {
+
+// ------------------------------------------------------------ basis tables
+// Host-side enumeration of the minimal symmetric basis (GPU path's own code).
+// Row order: degree-major p = 0..P-1, lexicographic tuples i_1<=...<=i_p.
+struct HostBasis {
+  int dK = 0, P = 0;
+  int64_t m = 0;
+  std::vector<uint8_t> degree;          // [m]
+  std::vector<uint8_t> ix;              // [m*3]; unused slots = dK (points at a 1.0)
+  std::vector<double> weight;           // [m]  1/sqrt(alpha! * dK^(p/2))
+};
+HostBasis build_host_basis(int dK, int P);
+int64_t count_basis(int dK, int P);  // m, or -1
+
+// Device copy of the tables in the packed form the kernels read.
+//   idx[r] = i1 | i2 << 8 | i3 << 16 | degree << 24  (unused slots = dK)
+//   w[r]   = fp32 weight
+struct DeviceBasis {
+  int dK = 0, P = 0;
+  int64_t m = 0;
+  uint32_t *idx = nullptr;
+  float *w = nullptr;
+  // Tensor-core tile order (dK in {32, 64}, P == 4); null when not built.
+  int n_tiles = 0;              // 64-feature tiles
+  int64_t m_pad = 0;            // n_tiles * 64
+  uint32_t *tile_desc = nullptr;  // [n_tiles] packed tile descriptors
+  int32_t *tile_row = nullptr;    // [m_pad] lexicographic row of each padded feature (-1 = pad)
+};
+
+// Returns the cached tables for the current device (builds them on first use).
+// Thread-safe.  Returns nullptr with *status set on failure.
+const DeviceBasis *get_device_basis(int dK, int P, int *status);
+
+// Per-(device, stream) grow-only scratch workspace.  Thread-safe.
+void *get_workspace(cudaStream_t stream, size_t bytes, int *status);
+
+// Device error word (first device-side failure code; 0 = none).
+int read_and_clear_device_error();
+int *device_error_ptr();
+
+// ------------------------------------------------------------ launchers
+int launch_prefill_simt(const void *q, const void *k, const void *v, float *out,
+                        float *state, int B, int H, int N, int dK, int dV, int P,
+                        bool bf16, const DeviceBasis *basis, cudaStream_t stream);
+
+int launch_decode(const void *q, const void *k, const void *v, float *state, float *out,
+                  int B, int H, int dK, int dV, int P, bool bf16,
+                  const DeviceBasis *basis, cudaStream_t stream);
+
+// ------------------------------------------------------------ profiling hook
+enum KernelId {
+  K_SIMT_CHUNK_STATES = 1,
+  K_SIMT_READOUT = 2,
+  K_DECODE_STREAM = 3,
+  K_DECODE_FINALIZE = 4,
+  K_TC_CHUNK_STATES = 5,
+  K_TC_READOUT = 6,
+  K_TC_PREP = 7,
+};
+void prof_call_begin();                          // start of an entry-point call
+void prof_kernel_begin(cudaStream_t s, int id);  // before a launch
+void prof_kernel_end(cudaStream_t s);            // after a launch
+
+// Status from the last CUDA call / launch.
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? SATA_OK : SATA_ERR_CUDA; }
+
+}  // namespace sata

@@ -36,6 +36,7 @@ from .sata import (
     taylor_kernel,
     feature_map,
     quadratic_form,
+    conditioning,
     feature_form,
     decode_step,
     final_state,
@@ -46,7 +47,7 @@ from .sata import (
 
 __all__ = [
     "basis_rows", "basis_weights", "basis_all", "multiplicity_factorial",
-    "taylor_kernel", "feature_map", "quadratic_form", "feature_form",
+    "taylor_kernel", "feature_map", "quadratic_form", "conditioning", "feature_form",
     "decode_step", "final_state", "softmax_attention", "basis_total",
     "flops_per_token_counted",
 ]

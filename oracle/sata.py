@@ -95,6 +95,25 @@ def quadratic_form(q, k, v, P: int, row_block: int = 1024):
     return num, den, num / den[..., None]
 
 
+def conditioning(q, k, P: int, row_block: int = 1024) -> np.ndarray:
+    """sum_{j<=i} |T_P(s_ij)| per row [B,H,N]: the scale against which rounding
+    in den_i = sum_{j<=i} T_P(s_ij) is measured (T_P is negative for some s
+    when P is even, so den_i can be much smaller than this sum)."""
+    q, k = _f64(q), _f64(k)
+    B, H, N, dK = q.shape
+    scale = 1.0 / math.sqrt(dK)
+    out = np.zeros((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            for i0 in range(0, N, row_block):
+                i1 = min(N, i0 + row_block)
+                s = (q[b, h, i0:i1] @ k[b, h, :i1].T) * scale
+                t = np.abs(taylor_kernel(s, P))
+                mask = np.arange(i1)[None, :] <= np.arange(i0, i1)[:, None]
+                out[b, h, i0:i1] = np.where(mask, t, 0.0).sum(axis=1)
+    return out
+
+
 def feature_form(q, k, v, P: int, state0=None):
     """Form (b): the per-token procedure of [SATA-eng] "恒定计算成本的工程实现".
 

@@ -1,0 +1,174 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle on the
+seeded workloads, plus edge cases.  Needs a B200."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import linear_cost_attention_b200 as sata
+from sata_inputs import WORKLOADS, DecodeStream, make_qkv, workload_inputs
+from tests.parity import TOL, out_row_error, state_col_error
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from linear_cost_attention_b200 import build
+
+    build.build()
+    torch.cuda.set_device(0)
+    yield
+    assert sata.sata_get_error() == sata.SATA_OK
+
+
+def gpu_prefill(q, k, v, P):
+    out, state = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P)
+    torch.cuda.synchronize()
+    return out.cpu().double().numpy(), state.cpu().double().numpy()
+
+
+def check_prefill(q, k, v, P, tol, heads=None, with_state=True):
+    out, state = gpu_prefill(q, k, v, P)
+    if heads is not None:  # oracle on a sample of (b, h) heads
+        sel = [(b, h) for b, h in heads]
+        qs = torch.stack([q[b, h] for b, h in sel])[None]
+        ks = torch.stack([k[b, h] for b, h in sel])[None]
+        vs = torch.stack([v[b, h] for b, h in sel])[None]
+        out = np.stack([out[b, h] for b, h in sel])[None]
+        state = np.stack([state[b, h] for b, h in sel])[None]
+        q, k, v = qs, ks, vs
+    num, den, ref = oracle.quadratic_form(q, k, v, P)
+    cond = oracle.conditioning(q, k, P)
+    err, excluded = out_row_error(out, ref, den, cond)
+    assert excluded <= max(4, out.shape[-2] * out.shape[0] * out.shape[1] // 200), excluded
+    assert err <= tol, (err, tol)
+    serr = None
+    if with_state:
+        S_ref = oracle.final_state(k, v, P)
+        serr = state_col_error(state, S_ref)
+        assert serr <= tol, (serr, tol)
+        # the degree-0 normaliser entry counts tokens exactly
+        assert np.all(state[..., 0, -1] == q.shape[2])
+    return err, serr, excluded
+
+
+def test_workload1_tiny_fp32_full():
+    q, k, v = workload_inputs(1)
+    out, state = gpu_prefill(q, k, v, 4)
+    assert out.shape == (1, 1, 64, 8) and state.shape == (1, 1, 165, 9)
+    num, den, ref, S_ref = oracle.feature_form(q, k, v, 4)
+    err, _ = out_row_error(out, ref, den, oracle.conditioning(q, k, 4))
+    assert err <= TOL["f32"]
+    assert state_col_error(state, S_ref) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("P", [4, 3, 2])
+def test_workload2_fp32(P):
+    q, k, v = workload_inputs(2)
+    check_prefill(q, k, v, P, TOL["f32"])
+
+
+def test_workload3_bf16():
+    q, k, v = workload_inputs(3)
+    check_prefill(q, k, v, 4, TOL["bf16"])
+
+
+def test_workload4_bf16_sampled_heads():
+    q, k, v = workload_inputs(4)
+    check_prefill(q, k, v, 4, TOL["bf16"], heads=[(0, 0), (0, 5)])
+
+
+@pytest.mark.parametrize("B,H,N,dK,dV,P,dt", [
+    (1, 1, 1, 8, 8, 4, "f32"),          # a single token
+    (1, 2, 77, 16, 8, 4, "f32"),        # ragged tail, dK != dV
+    (2, 3, 200, 8, 64, 3, "f32"),
+    (1, 1, 1000, 64, 16, 4, "f32"),     # several chunks + ragged tail
+    (3, 1, 129, 32, 32, 1, "f32"),      # P = 1: running mean
+    (1, 2, 300, 64, 64, 2, "bf16"),
+    (2, 2, 1100, 32, 32, 4, "bf16"),
+])
+def test_edge_shapes(B, H, N, dK, dV, P, dt):
+    q, k, v = make_qkv(B, H, N, dK, dV, seed=B * 1000 + N, dtype=dt)
+    check_prefill(q, k, v, P, TOL[dt])
+
+
+def test_invalid_call_raises():
+    q = torch.zeros(1, 1, 4, 8, device="cuda")
+    with pytest.raises(sata.SataError):
+        sata.prefill(q, q, q, P=5)
+    with pytest.raises(sata.SataError):
+        sata.sata_prefill(q, q, q, q, q, 1, 1, 4, 8, 8, 4, torch.float32)  # aliasing
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_prefill_then_decode_equals_longer_prefill(dt):
+    B, H, N0, t, dK, dV, P = 2, 2, 96, 6, 16, 16, 4
+    q, k, v = make_qkv(B, H, N0 + t, dK, dV, seed=31, dtype=dt)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    out_full, state_full = sata.prefill(qc, kc, vc, P)
+    _, state = sata.prefill(qc[:, :, :N0].contiguous(), kc[:, :, :N0].contiguous(),
+                            vc[:, :, :N0].contiguous(), P)
+    outs = []
+    for s in range(t):
+        i = N0 + s
+        outs.append(sata.decode_step(qc[:, :, i].contiguous(), kc[:, :, i].contiguous(),
+                                     vc[:, :, i].contiguous(), state, P).cpu())
+    torch.cuda.synchronize()
+    got = torch.stack(outs, dim=2).double().numpy()
+    num, den, ref = oracle.quadratic_form(q, k, v, P)
+    cond = oracle.conditioning(q, k, P)
+    err, _ = out_row_error(got, ref[:, :, N0:], den[:, :, N0:], cond[:, :, N0:])
+    assert err <= TOL[dt]
+    tol = TOL[dt]
+    assert state_col_error(state.cpu().double().numpy(), oracle.final_state(k, v, P)) <= tol
+    # decode continues the GPU prefill consistently with the GPU's longer prefill
+    assert state_col_error(state.cpu().double().numpy(),
+                           state_full.cpu().double().numpy()) <= 10 * TOL["f32"]
+
+
+def test_workload5_decode():
+    """Workload 5: bf16 prefill N=8192 for B=32,H=8 (dK=dV=64, P=4), then 1024
+    decode steps.  Oracle: two sampled heads over every step from the oracle's
+    own prefill state; all heads at steps 1, 512, 1024 from the GPU's state just
+    before the step."""
+    w = WORKLOADS[5]
+    P = w.P
+    q, k, v = workload_inputs(5)
+    sample = [(3, 1), (30, 6)]
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    _, state = sata.prefill(qc, kc, vc, P)
+    del qc, kc, vc
+    ks = torch.stack([k[b, h] for b, h in sample])[None]
+    vs = torch.stack([v[b, h] for b, h in sample])[None]
+    S_or = oracle.final_state(ks, vs, P)
+    st_gpu = torch.stack([state[b, h] for b, h in sample])[None].cpu().double().numpy()
+    assert state_col_error(st_gpu, S_or) <= TOL["bf16"]
+
+    stream = DecodeStream(5)
+    check_all = {1, 512, 1024}
+    worst = 0.0
+    for t in range(1, w.decode_steps + 1):
+        qt, kt, vt = stream.next()
+        if t in check_all:
+            before = state.cpu()
+        out = sata.decode_step(qt.cuda(), kt.cuda(), vt.cuda(), state, P)
+        o = out.cpu().double().numpy()
+        # sampled heads against the oracle's own trajectory
+        qs_ = np.stack([qt[b, h, 0].double().numpy() for b, h in sample])[None]
+        ks_ = np.stack([kt[b, h, 0].double().numpy() for b, h in sample])[None]
+        vs_ = np.stack([vt[b, h, 0].double().numpy() for b, h in sample])[None]
+        ref, S_or = oracle.decode_step(qs_, ks_, vs_, S_or, P)
+        got = np.stack([o[b, h] for b, h in sample])[None]
+        e = np.max(np.abs(got - ref), axis=-1) / np.max(np.abs(ref), axis=-1)
+        worst = max(worst, float(e.max()))
+        if t in check_all:  # every head, from the GPU state before this step
+            for b in range(w.B):
+                ref_b, _ = oracle.decode_step(qt[b:b + 1, :, 0], kt[b:b + 1, :, 0],
+                                              vt[b:b + 1, :, 0], before[b:b + 1], P)
+                eb = np.max(np.abs(o[b:b + 1] - ref_b), axis=-1) / np.max(np.abs(ref_b), axis=-1)
+                assert eb.max() <= TOL["bf16"], (t, b, eb.max())
+            del before
+    assert worst <= TOL["bf16"], worst
+    st_gpu = torch.stack([state[b, h] for b, h in sample])[None].cpu().double().numpy()
+    assert state_col_error(st_gpu, S_or) <= TOL["bf16"]
