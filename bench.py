@@ -461,6 +461,34 @@ def run_reference(args):
     }
 
 
+def profile_case(case: str):
+    """Small cases for ncu captures: a few launches of one kernel on inputs
+    larger than L2 but a few GB on the device at most."""
+    import torch
+
+    import linear_cost_attention_b200 as sata
+    from sata_inputs import make_qkv
+
+    torch.cuda.set_device(0)
+    if case == "decode":
+        B, H, N, d, P = 8, 8, 256, 64, 4          # state 797 MB (> L2)
+        q, k, v = make_qkv(B, H, N, d, d, seed=3, dtype="bf16")
+        _, state = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P)
+        for t in range(5):
+            qt, kt, vt = (x[:, :, t].contiguous().cuda() for x in (q, k, v))
+            sata.decode_step(qt, kt, vt, state, P)
+    elif case == "prefill":
+        B, H, N, d, P = 1, 2, 4096, 64, 4         # state 25 MB; chunk states > L2
+        q, k, v = make_qkv(B, H, N, d, d, seed=4, dtype="bf16")
+        qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+        for _ in range(3):
+            sata.prefill(qd, kd, vd, P)
+    else:
+        raise SystemExit(f"unknown profile case {case}")
+    torch.cuda.synchronize()
+    assert sata.sata_get_error() == sata.SATA_OK
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -470,7 +498,12 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=128)
     ap.add_argument("--ref-rows", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["decode", "prefill"], default=None,
+                    help="run a small case of one kernel for an ncu capture and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank = int(os.environ.get("RANK", "0"))
