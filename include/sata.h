@@ -100,6 +100,32 @@ int sata_decode_step(const void *q, const void *k, const void *v, float *state,
                      float *out, int B, int H, int dK, int dV, int P,
                      sata_dtype dt, sata_stream_t stream);
 
+/* sata_decode_step without any device allocation.  (The paper has no
+ * counterpart: this is an interface for callers that cannot allocate device
+ * memory: hosts whose caching allocator owns the whole GPU, serving loops
+ * that must not hit cudaMalloc/cudaFree because those can synchronise the
+ * device, plug-in hosts whose policy forbids library-side allocations.)
+ * Same arguments, layouts, semantics and results as sata_decode_step.  It
+ * calls no cudaMalloc, cudaFree or other allocating routine: its scratch (the
+ * per-head partial sums) is a file-scope __device__ array of
+ * SATA_NOALLOC_MAX_PARTIALS floats (256 KiB), and its basis tables are static
+ * __device__ arrays as well; every GPU that loads the library holds both
+ * until the process exits.
+ *   - B*H*(dV+1) > SATA_NOALLOC_MAX_PARTIALS (e.g. more than 1008 heads at
+ *     dV = 64) -> SATA_ERR_INVALID_ARG, nothing launched.
+ *   - The first call on a device does a one-time set-up with that device
+ *     current (resolves the arrays' device addresses with
+ *     cudaGetSymbolAddress and copies the basis tables in, synchronously);
+ *     make that first call before any stream capture.
+ *   - All calls on a device share the scratch, which keeps the last call's
+ *     contents; each call clears what it uses first.  Calls that overlap on
+ *     the GPU (other streams or host threads) race on it: order them. */
+#define SATA_NOALLOC_MAX_PARTIALS 65536
+int sata_decode_step_noalloc(const void *q, const void *k, const void *v,
+                             float *state, float *out, int B, int H, int dK,
+                             int dV, int P, sata_dtype dt,
+                             sata_stream_t stream);
+
 /* Synchronises `stream`, then reports (and clears) the first device-side error
  * recorded by this library's kernels on the current device (a bounded wait
  * that gave up -> SATA_ERR_TIMEOUT) or a pending CUDA error (-> SATA_ERR_CUDA).

@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
     L.sata_status_string.restype = ctypes.c_char_p
     L.sata_release.argtypes = []
     L.sata_release.restype = None
+    L.sata_decode_step_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    L.sata_decode_step_noalloc.restype = i
     L.sata_profile_enable.argtypes = [i]
     L.sata_profile_enable.restype = i
     L.sata_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(i), i]
@@ -131,6 +133,15 @@ def sata_decode_step(q, k, v, state, out, B, H, dK, dV, P, dtype, stream=None) -
                                 dV, P, _dtype_code(dtype), _stream(stream))
     if st != SATA_OK:
         raise SataError(st, "sata_decode_step")
+
+
+def sata_decode_step_noalloc(q, k, v, state, out, B, H, dK, dV, P, dtype, stream=None) -> None:
+    """sata_decode_step for callers that cannot allocate device memory: its
+    scratch and tables are static device arrays (limit B*H*(dV+1) <= 65536)."""
+    st = lib().sata_decode_step_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), B, H,
+                                        dK, dV, P, _dtype_code(dtype), _stream(stream))
+    if st != SATA_OK:
+        raise SataError(st, "sata_decode_step_noalloc")
 
 
 def sata_get_error(stream=None) -> int:

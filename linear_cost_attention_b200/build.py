@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsata.so")
 
-SOURCES = ["sata_abi.cu", "basis.cpp", "prefill_simt.cu", "decode.cu"]
+SOURCES = ["sata_abi.cu", "basis.cpp", "prefill_simt.cu", "decode.cu", "decode_noalloc.cu"]
 HEADERS = ["sata_internal.h", "common.cuh"]
 
 NVCC_FLAGS = [

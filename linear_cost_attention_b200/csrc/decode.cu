@@ -200,3 +200,52 @@ int launch_decode(const void *q, const void *k, const void *v, float *state, flo
 }
 
 }  // namespace sata
+
+namespace sata {
+namespace {
+
+// Same two kernels as run_decode, with the basis tables and the partial-sum
+// scratch supplied by the caller instead of the library's caches.
+template <int D1, typename T>
+int run_decode_scratch(const void *q, const void *k, const void *v, float *state, float *out,
+                       int BH, int dK, const uint32_t *idx, const float *w, int64_t m, float *y,
+                       cudaStream_t stream) {
+  constexpr int NT = D1 * DecodeShape<D1>::KB;
+  constexpr long long L = 4LL * NT * kIters;
+  const long long E = (long long)BH * m * D1;
+  if (cudaMemsetAsync(y, 0, (size_t)BH * D1 * sizeof(float), stream) != cudaSuccess)
+    return SATA_ERR_CUDA;
+  const long long blocks = (E + L - 1) / L;
+  if (blocks > 0x7fffffffLL) return SATA_ERR_INVALID_ARG;
+  decode_stream<D1, T><<<(unsigned)blocks, NT, 0, stream>>>(
+      (const T *)q, (const T *)k, (const T *)v, state, idx, w, (int)m, dK, E, y);
+  const int n = BH * (D1 - 1);
+  decode_finalize<D1><<<(n + 255) / 256, 256, 0, stream>>>(y, out, BH);
+  return cuda_status(cudaGetLastError());
+}
+
+template <typename T>
+int dispatch_scratch(int dK, int dV, const void *q, const void *k, const void *v, float *state,
+                     float *out, int BH, const uint32_t *idx, const float *w, int64_t m,
+                     float *y, cudaStream_t s) {
+  switch (dV) {
+    case 8: return run_decode_scratch<9, T>(q, k, v, state, out, BH, dK, idx, w, m, y, s);
+    case 16: return run_decode_scratch<17, T>(q, k, v, state, out, BH, dK, idx, w, m, y, s);
+    case 32: return run_decode_scratch<33, T>(q, k, v, state, out, BH, dK, idx, w, m, y, s);
+    case 64: return run_decode_scratch<65, T>(q, k, v, state, out, BH, dK, idx, w, m, y, s);
+  }
+  return SATA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+int launch_decode_scratch(const void *q, const void *k, const void *v, float *state, float *out,
+                          int B, int H, int dK, int dV, bool bf16, const uint32_t *idx,
+                          const float *w, int64_t m, float *y, cudaStream_t stream) {
+  const int BH = B * H;
+  if (bf16)
+    return dispatch_scratch<__nv_bfloat16>(dK, dV, q, k, v, state, out, BH, idx, w, m, y, stream);
+  return dispatch_scratch<float>(dK, dV, q, k, v, state, out, BH, idx, w, m, y, stream);
+}
+
+}  // namespace sata

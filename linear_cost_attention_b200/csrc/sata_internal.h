@@ -60,6 +60,12 @@ int launch_decode(const void *q, const void *k, const void *v, float *state, flo
                   int B, int H, int dK, int dV, int P, bool bf16,
                   const DeviceBasis *basis, cudaStream_t stream);
 
+// Decode with caller-supplied basis tables (packed as in DeviceBasis) and
+// partial-sum scratch y of at least B*H*(dV+1) floats.
+int launch_decode_scratch(const void *q, const void *k, const void *v, float *state, float *out,
+                          int B, int H, int dK, int dV, bool bf16, const uint32_t *idx,
+                          const float *w, int64_t m, float *y, cudaStream_t stream);
+
 // ------------------------------------------------------------ profiling hook
 enum KernelId {
   K_SIMT_CHUNK_STATES = 1,
