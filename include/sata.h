@@ -79,9 +79,10 @@ int64_t sata_index_table(int dK, int p, int32_t *host_out, int64_t cap_elems);
 /* Causal prefill from a zero state.  Writes out (every token) and overwrites
  * state with S after the last token.  q, k, v, out, state: see layouts above;
  * out and state must not overlap each other or the inputs.
- * The bf16 path computes the feature products in fp32, rounds features, the
- * chunk-boundary states and the in-chunk Taylor scores to bf16 for the tensor
- * cores, and accumulates in fp32; the fp32 path stays in fp32 throughout.
+ * Paths: bf16 inputs with dK = dV = 64 and P = 4 run on the tcgen05 tensor
+ * cores (features and chunk-boundary states rounded to bf16, in-chunk Taylor
+ * scores split into bf16 hi + lo parts, fp32 accumulation); every other
+ * supported case runs in fp32 on CUDA cores.
  * Returns SATA_OK, SATA_ERR_INVALID_ARG, SATA_ERR_UNSUPPORTED, SATA_ERR_NOMEM
  * or SATA_ERR_CUDA. */
 int sata_prefill(const void *q, const void *k, const void *v, float *out,

@@ -13,8 +13,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsata.so")
 
-SOURCES = ["sata_abi.cu", "basis.cpp", "prefill_simt.cu", "decode.cu", "decode_noalloc.cu"]
-HEADERS = ["sata_internal.h", "common.cuh"]
+SOURCES = ["sata_abi.cu", "basis.cpp", "tile_order.cu", "prefill_simt.cu", "prefill_tc.cu",
+           "decode.cu", "decode_noalloc.cu"]
+HEADERS = ["sata_internal.h", "common.cuh", "tc_common.cuh", "tile_gen.cuh", "tile_order.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -24,6 +24,7 @@ namespace sata {
 namespace {
 
 constexpr int kIters = 16;  // iterations (of 4*NT elements) per block
+constexpr int kUnroll = 4;  // iterations whose loads are in flight together
 
 template <int D1> struct DecodeShape;
 template <> struct DecodeShape<65> { static constexpr int KB = 4; };   // 260 threads
@@ -96,39 +97,49 @@ __global__ void __launch_bounds__(D1 *DecodeShape<D1>::KB)
     acc[u] = 0.f;
   };
 
-  for (int it = 0; it < kIters; ++it) {
-    const long long e = e_begin + (long long)it * PER_IT + 4 * tid;
-    if (e >= e_end) break;
-    const int rbase = it * ROWS_IT;
-    float s[4];
-    const bool full = (e + 3 < e_end);
-    if (full) {
-      const float4 x = __ldcs(reinterpret_cast<const float4 *>(state + e));
-      s[0] = x.x; s[1] = x.y; s[2] = x.z; s[3] = x.w;
-    } else {
+  // kUnroll iterations at a time: all their 16-byte loads are issued before any
+  // is used, so each thread keeps kUnroll*16 bytes in flight.
+  for (int it0 = 0; it0 < kIters; it0 += kUnroll) {
+    float s[kUnroll][4];
+    long long e[kUnroll];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) s[u] = (e + u < e_end) ? state[e + u] : 0.f;
-    }
+    for (int j = 0; j < kUnroll; ++j) {
+      e[j] = e_begin + (long long)(it0 + j) * PER_IT + 4 * tid;
+      if (e[j] + 3 < e_end) {
+        const float4 x = __ldcs(reinterpret_cast<const float4 *>(state + e[j]));
+        s[j][0] = x.x; s[j][1] = x.y; s[j][2] = x.z; s[j][3] = x.w;
+      } else {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (!full && e + u >= e_end) continue;  // past the end of the array
-      const int rr = rbase + rof[u];
-      const int bh = s_bh[min(rr, nrows - 1)];
-      if (bh != cur[u]) {
-        flush(u);
-        cur[u] = bh;
-        vv[u] = (col[u] < DV) ? to_f32(v[(size_t)bh * DV + col[u]]) : 1.f;
+        for (int u = 0; u < 4; ++u) s[j][u] = (e[j] + u < e_end) ? state[e[j] + u] : 0.f;
       }
-      const float sn = fmaf(s_fk[min(rr, nrows - 1)], vv[u], s[u]);
-      s[u] = sn;
-      acc[u] = fmaf(s_fq[min(rr, nrows - 1)], sn, acc[u]);
     }
-    if (full) {
-      __stcs(reinterpret_cast<float4 *>(state + e), make_float4(s[0], s[1], s[2], s[3]));
-    } else {
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (e + u < e_end) state[e + u] = s[u];
+    for (int j = 0; j < kUnroll; ++j) {
+      if (e[j] >= e_end) break;
+      const bool full = (e[j] + 3 < e_end);
+      const int rbase = (it0 + j) * ROWS_IT;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (!full && e[j] + u >= e_end) continue;  // past the end of the array
+        const int rr = min(rbase + rof[u], nrows - 1);
+        const int bh = s_bh[rr];
+        if (bh != cur[u]) {
+          flush(u);
+          cur[u] = bh;
+          vv[u] = (col[u] < DV) ? to_f32(v[(size_t)bh * DV + col[u]]) : 1.f;
+        }
+        const float sn = fmaf(s_fk[rr], vv[u], s[j][u]);
+        s[j][u] = sn;
+        acc[u] = fmaf(s_fq[rr], sn, acc[u]);
+      }
+      if (full) {
+        __stcs(reinterpret_cast<float4 *>(state + e[j]),
+               make_float4(s[j][0], s[j][1], s[j][2], s[j][3]));
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (e[j] + u < e_end) state[e[j] + u] = s[j][u];
+      }
     }
   }
 #pragma unroll

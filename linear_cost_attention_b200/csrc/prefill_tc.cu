@@ -1,0 +1,691 @@
+// Tensor-core (tcgen05) prefill for bf16 inputs with dK = dV = 64, P = 4.
+//
+// Same chunked decomposition as the CUDA-core path (prefill_simt.cu), with
+// both state contractions on the 5th-generation tensor cores:
+//
+//   tc_chunk_states  one CTA per (head, 4 x 128 basis rows): the four state
+//     tiles S[128 x 80] (dV+1 = 65 columns padded to the MMA's N = 80) stay in
+//     TMEM for the whole sequence.  Per 64 tokens: TMA brings K and V; eight
+//     generator warps write phi(K)^T (basis rows x tokens, MN-major) into
+//     shared memory, one thread per token; one thread issues
+//     S += phi(K)^T [V, 1] (M = 128, N = 80, K = 16 per instruction).  At every
+//     chunk boundary the epilogue warps copy S to a bf16 snapshot (the state
+//     before the next chunk, "恒定计算成本的工程实现": the fixed-size state), and
+//     after the last token write the fp32 state in lexicographic row order.
+//   tc_readout       one CTA per (head, 128 tokens of chunk c):
+//     D[128 x 80] = sum over 750 tiles of 64 basis rows of phi(Q_tile) S_(c-1)
+//     (phi(Q) generated per tile into shared memory, snapshot tiles streamed by
+//     TMA), plus the in-chunk part sum_{c0 <= j <= i} T_4(s_ij) [v_j, 1] per
+//     64-key block: scores Q K^T into TMEM, T_4 and the causal mask by the
+//     epilogue warps, P split into bf16 hi + lo parts (T_4 rounded to bf16 loses
+//     too much on rows whose denominator cancels), P_hi [V, 1] + P_lo [V, 1]
+//     into D; out = D[:, :64] / D[:, 64].
+//
+// Warp roles (512 threads): 0 TMA producer, 1 MMA issuer (one thread) and TMEM
+// owner, 2 second TMA producer (readout), 4-7 epilogue (TMEM lane quarters),
+// 8-15 feature generators.  Every mbarrier wait is bounded (tc_common.cuh);
+// on a timeout the kernel records an error, drains what it issued and frees
+// its TMEM before returning.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "sata_internal.h"
+#include "tc_common.cuh"
+#include "tile_gen.cuh"
+#include "tile_order.h"
+
+namespace sata {
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 512;
+constexpr int kNP = 80;             // MMA N for [V, 1]: dV + 1 = 65 rounded up to 16
+constexpr uint32_t kRow = 128;      // bytes per 64-element bf16 row
+constexpr uint32_t kOne = 0x3F80u;  // bf16 1.0
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+  const uint32_t a = smem_u32(p);
+  return p + (((a + 1023u) & ~1023u) - a);
+}
+
+// [V, 1] second column block: row r holds 1.0 at column 64 (logical chunk 0,
+// element 0), zeros elsewhere, in the 128-byte-swizzled layout.
+__device__ __forceinline__ void fill_ones(uint8_t *blk, int rows) {
+  for (int i = threadIdx.x; i < rows * 8; i += blockDim.x) {
+    const int r = i >> 3, c = i & 7;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (c == (r & 7)) v.x = kOne;
+    *reinterpret_cast<uint4 *>(blk + r * kRow + c * 16) = v;
+  }
+}
+
+// ============================================================ chunk states
+constexpr int kUF = 4;                               // 128-row state tiles per item
+constexpr int kUT = 64;                              // tokens per step
+constexpr uint32_t kUTileBytes = kUT * kRow;         // 64 rows x 64 tokens: 8 KiB
+constexpr uint32_t kUAStage = 2 * kUF * kUTileBytes;  // 64 KiB
+constexpr uint32_t kUKV = kUT * kRow;                // 8 KiB
+constexpr uint32_t kUOffA = 0, kUOffK = 2 * kUAStage, kUOffV = kUOffK + 2 * kUKV,
+                   kUOffOnes = kUOffV + 2 * kUKV, kUOffBar = kUOffOnes + kUKV;
+constexpr uint32_t kUSmem = kUOffBar + 256 + 1024;
+
+struct UParams {
+  const TileDesc *tiles;
+  const int32_t *row_of_slot;
+  GenWeights W;
+  int n_tiles;  // even
+  int N, C, nsnap, m, m_pad, n_batches, n_items, head0;
+  __nv_bfloat16 *snap;  // [G][nsnap][65][m_pad]
+  float *state;         // [BH][m][65]
+  int *err;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_chunk_states(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const UParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *sA = smem + kUOffA, *sK = smem + kUOffK, *sV = smem + kUOffV, *sOnes = smem + kUOffOnes;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kUOffBar);
+  uint64_t *kv_full = bar, *kv_empty = bar + 2, *a_full = bar + 4, *a_empty = bar + 6,
+           *snap_full = bar + 8, *snap_done = bar + 9, *drain = bar + 13;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 14);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 15);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1 + 8);
+      mbar_init(&a_full[s], 8);
+      mbar_init(&a_empty[s], 1);
+    }
+    mbar_init(snap_full, 1);
+    for (int f = 0; f < kUF; ++f) mbar_init(&snap_done[f], 4);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  fill_ones(sOnes, kUT);
+  fence_proxy_async_smem();
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int nsub = (p.N + kUT - 1) / kUT;
+  const int sub_per_chunk = p.C / kUT;
+  const int n_mt = p.n_tiles / 2;
+
+  if (warp == 0) {
+    // ---------------- TMA producer: K and V rows of 64 tokens
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int bh = p.head0 + item / p.n_batches;
+        for (int s = 0; s < nsub; ++s, ++it) {
+          const int st = it & 1;
+          if (it >= 2 && !(ok = mbar_wait(&kv_empty[st], ((it >> 1) - 1) & 1, abort_flag, p.err)))
+            break;
+          mbar_arrive_expect_tx(&kv_full[st], 2 * kUKV);
+          tma_load_3d(sK + st * kUKV, &tmK, &kv_full[st], 0, s * kUT, bh);
+          tma_load_3d(sV + st * kUKV, &tmV, &kv_full[st], 0, s * kUT, bh);
+        }
+      }
+      // let the loads already issued land before the CTA can exit
+      for (uint32_t j = it > 2 ? it - 2 : 0; j < it; ++j) {
+        volatile int never = 0;
+        mbar_wait(&kv_full[j & 1], (j >> 1) & 1, &never, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kNP, true, true);
+      uint32_t it = 0, events = 0;
+      bool after_event = false;  // the epilogue must release each tile first
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int batch = item % p.n_batches;
+        const int nmt = min(kUF, n_mt - batch * kUF);
+        for (int s = 0; ok && s < nsub; ++s, ++it) {
+          const int st = it & 1;
+          const uint32_t ph = (it >> 1) & 1;
+          if (!(ok = mbar_wait(&kv_full[st], ph, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&a_full[st], ph, abort_flag, p.err))) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + st * kUAStage);
+          const uint32_t v0 = smem_u32(sV + st * kUKV);
+          const uint32_t lbo_b = smem_u32(sOnes) - v0;
+          for (int f = 0; f < kUF; ++f) {
+            // every tile's barrier is waited once per event, in order, so no
+            // barrier can run two phases ahead of its waiter
+            if (after_event) {
+              if (!(ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err))) break;
+              tc_fence_after();
+            }
+            if (f >= nmt) continue;
+#pragma unroll
+            for (int k = 0; k < kUT / 16; ++k) {
+              const uint64_t ad = smem_desc_sw128(a0 + 2 * f * kUTileBytes + k * 2048,
+                                                  kUTileBytes, 1024);
+              const uint64_t bd = smem_desc_sw128(v0 + k * 2048, lbo_b, 1024);
+              mma_bf16_ss(tmem + f * kNP, ad, bd, idesc, (s > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          after_event = false;
+          mma_commit(&a_empty[st]);
+          mma_commit(&kv_empty[st]);
+          const bool boundary = ((s + 1) % sub_per_chunk == 0) && (s + 1 < nsub);
+          if (boundary || s == nsub - 1) {
+            mma_commit(snap_full);
+            ++events;
+            after_event = true;
+          }
+        }
+      }
+      // every MMA issued so far completes before the TMEM is released
+      mma_commit(drain);
+      volatile int never = 0;
+      mbar_wait(drain, 0, &never, p.err);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- epilogue: snapshots and final state
+    const int q4 = warp & 3;
+    const int row = 32 * q4 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
+    uint32_t events = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int hb = item / p.n_batches, batch = item % p.n_batches;
+      const int nmt = min(kUF, n_mt - batch * kUF);
+      for (int s = 0; s < nsub; ++s) {
+        const bool boundary = ((s + 1) % sub_per_chunk == 0) && (s + 1 < nsub);
+        if (!boundary && s != nsub - 1) continue;
+        if (!(ok = mbar_wait(snap_full, events & 1, abort_flag, p.err))) break;
+        ++events;
+        tc_fence_after();
+        for (int f = 0; f < kUF; ++f) {
+          uint32_t v[kNP];
+          if (f < nmt) {
+#pragma unroll
+            for (int j = 0; j < kNP / 16; ++j)
+              tmem_ld16(tl + f * kNP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+            tmem_ld_wait();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&snap_done[f]);
+          if (f >= nmt) continue;
+          const int slot = (batch * kUF + f) * 128 + row;
+          if (boundary) {
+            const int c = (s + 1) / sub_per_chunk - 1;
+            __nv_bfloat16 *dst =
+                p.snap + ((size_t)(hb * p.nsnap + c) * 65) * p.m_pad + slot;
+#pragma unroll
+            for (int n = 0; n < 65; ++n)
+              dst[(size_t)n * p.m_pad] = __float2bfloat16_rn(__uint_as_float(v[n]));
+          } else {
+            const int r = p.row_of_slot[slot];
+            if (r >= 0) {
+              float *dst = p.state + ((size_t)(p.head0 + hb) * p.m + r) * 65;
+#pragma unroll
+              for (int n = 0; n < 65; ++n) dst[n] = __uint_as_float(v[n]);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // ---------------- feature generators: phi(K)^T tiles, one thread per token
+    const int gw = warp - 8;
+    const int t = lane + 32 * (gw & 1);
+    const int fq = gw >> 1;  // feature tiles fq and fq + 4 of the item
+    uint32_t it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int batch = item % p.n_batches;
+      const int tile0 = batch * 2 * kUF;
+      for (int s = 0; s < nsub; ++s, ++it) {
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (!(ok = mbar_wait(&kv_full[st], ph, abort_flag, p.err))) break;
+        if (it >= 2 && !(ok = mbar_wait(&a_empty[st], ph ^ 1, abort_flag, p.err))) break;
+        const uint8_t *krow = sK + st * kUKV + t * kRow;
+        const bool valid = s * kUT + t < p.N;
+#pragma unroll 1
+        for (int j = fq; j < 2 * kUF; j += 4) {
+          const int ft = tile0 + j;
+          uint32_t out[32];
+          if (valid && ft < p.n_tiles) {
+            const TileDesc td = p.tiles[ft];
+            gen_tile(td, krow, (uint32_t)(t & 7), p.W, out);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) out[q] = 0u;
+          }
+          store_tile_row(sA + st * kUAStage + j * kUTileBytes, (uint32_t)t, out);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&a_full[st]);
+          mbar_arrive(&kv_empty[st]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ============================================================ readout
+constexpr int kRStages = 4;
+constexpr int kKB = 64;                  // keys per in-chunk block
+constexpr uint32_t kRTile = 128 * kRow;  // 128 tokens x 64 features: 16 KiB
+constexpr uint32_t kRB = kNP * kRow;     // 80 x 64 snapshot tile: 10 KiB
+constexpr uint32_t kRKV = kKB * kRow;    // 64 keys x 64: 8 KiB
+constexpr uint32_t kROffQ = 0, kROffA = kROffQ + kRTile, kROffB = kROffA + kRStages * kRTile,
+                   kROffK = kROffB + kRStages * kRB, kROffV = kROffK + kRKV,
+                   kROffOnes = kROffV + kRKV, kROffP = kROffOnes + kRKV,
+                   kROffBar = kROffP + 2 * kRTile;
+constexpr uint32_t kRSmem = kROffBar + 256 + 1024;
+
+struct RParams {
+  const TileDesc *tiles;
+  GenWeights W;
+  int n_tiles;
+  int N, C, nsnap, head0;
+  float *out;  // [BH][N][64]
+  int *err;
+};
+
+__device__ __forceinline__ float taylor4(float s) {
+  return fmaf(fmaf(fmaf(s, 1.0f / 6.0f, 0.5f), s, 1.0f), s, 1.0f);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_readout(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
+               const RParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *sQ = smem + kROffQ, *sA = smem + kROffA, *sB = smem + kROffB, *sK = smem + kROffK,
+          *sV = smem + kROffV, *sOnes = smem + kROffOnes, *sP = smem + kROffP;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kROffBar);
+  uint64_t *q_full = bar, *kv_full = bar + 1, *kv_empty = bar + 2, *s_full = bar + 3,
+           *p_full = bar + 4, *o_full = bar + 5, *a_full = bar + 6, *a_empty = bar + 10,
+           *b_full = bar + 14, *b_empty = bar + 18;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 22);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 23);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * 128;
+  const int hrel = blockIdx.y;
+  const int bh = p.head0 + hrel;
+  const int chunk = t0 / p.C;
+  const int c0 = chunk * p.C;
+  const int nkb = (t0 - c0) / kKB + 128 / kKB;  // key blocks from the chunk start through t0+127
+  const bool inter = chunk > 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(o_full, 1);
+    for (int s = 0; s < kRStages; ++s) {
+      mbar_init(&a_full[s], 4);
+      mbar_init(&a_empty[s], 1);
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  fill_ones(sOnes, kKB);
+  fence_proxy_async_smem();
+  if (warp == 1) tmem_alloc(tmem_slot, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tD = tmem, tS = tmem + 128;
+
+  if (warp == 0) {
+    // ---------------- TMA producer: snapshot tiles S_(c-1)[80 x 64 rows]
+    if (lane == 0 && inter) {
+      prefetch_tensormap(&tmS);
+      int i = 0;
+      for (; i < p.n_tiles; ++i) {
+        const int st = i % kRStages;
+        if (i >= kRStages &&
+            !mbar_wait(&b_empty[st], ((i / kRStages) - 1) & 1, abort_flag, p.err))
+          break;
+        mbar_arrive_expect_tx(&b_full[st], kRB);
+        tma_load_3d(sB + st * kRB, &tmS, &b_full[st], 64 * i, 0, hrel * p.nsnap + chunk - 1);
+      }
+      for (int j = max(0, i - kRStages); j < i; ++j) {
+        volatile int never = 0;
+        mbar_wait(&b_full[j % kRStages], (j / kRStages) & 1, &never, p.err);
+      }
+    }
+  } else if (warp == 2) {
+    // ---------------- TMA producer: Q once, then K, V blocks of the chunk
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      mbar_arrive_expect_tx(q_full, kRTile);
+      tma_load_3d(sQ, &tmQ, q_full, 0, t0, bh);
+      int kb = 0;
+      for (; kb < nkb; ++kb) {
+        if (kb > 0 && !mbar_wait(kv_empty, (kb - 1) & 1, abort_flag, p.err)) break;
+        mbar_arrive_expect_tx(kv_full, 2 * kRKV);
+        tma_load_3d(sK, &tmK, kv_full, 0, c0 + kKB * kb, bh);
+        tma_load_3d(sV, &tmV, kv_full, 0, c0 + kKB * kb, bh);
+      }
+      volatile int never = 0;
+      mbar_wait(q_full, 0, &never, p.err);
+      if (kb > 0) mbar_wait(kv_full, (kb - 1) & 1, &never, p.err);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_inter = idesc_bf16_f32(128, kNP, false, false);
+      constexpr uint32_t id_qk = idesc_bf16_f32(128, kKB, false, false);
+      constexpr uint32_t id_pv = idesc_bf16_f32(128, kNP, false, true);
+      bool d_init = false, ok = true;
+      int kb_qk = 0, kb_pv = 0;
+      const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV);
+      const uint32_t p0 = smem_u32(sP), lbo_v = smem_u32(sOnes) - v0;
+      ok = mbar_wait(q_full, 0, abort_flag, p.err);
+      // in-chunk part, advanced whenever its inputs are ready
+      auto intra = [&](bool block) {
+        while (ok && kb_pv < nkb) {
+          if (kb_qk == kb_pv) {  // next: scores of block kb_qk
+            if (block) {
+              if (!(ok = mbar_wait(kv_full, kb_qk & 1, abort_flag, p.err))) return;
+            } else if (!mbar_try_wait(kv_full, kb_qk & 1)) {
+              return;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_bf16_ss(tS, smem_desc_sw128(q0 + 32 * k, 16, 1024),
+                          smem_desc_sw128(k0 + 32 * k, 16, 1024), id_qk, k > 0 ? 1u : 0u);
+            mma_commit(s_full);
+            ++kb_qk;
+          } else {  // next: P [V, 1] of block kb_pv
+            if (block) {
+              if (!(ok = mbar_wait(p_full, kb_pv & 1, abort_flag, p.err))) return;
+            } else if (!mbar_try_wait(p_full, kb_pv & 1)) {
+              return;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 2 * (kKB / 16); ++k) {  // hi part, then lo part
+              const int kk = k % (kKB / 16);
+              const uint64_t ad = smem_desc_sw128(p0 + (k / (kKB / 16)) * kRTile + 32 * kk, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(v0 + kk * 2048, lbo_v, 1024);
+              mma_bf16_ss(tD, ad, bd, id_pv, (d_init || k > 0) ? 1u : 0u);
+            }
+            d_init = true;
+            mma_commit(kv_empty);
+            ++kb_pv;
+          }
+        }
+      };
+      if (ok) intra(false);
+      if (ok && inter) {
+        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+        for (int i = 0; i < p.n_tiles; ++i) {
+          const int st = i % kRStages;
+          const uint32_t ph = (i / kRStages) & 1;
+          if (!(ok = mbar_wait(&a_full[st], ph, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&b_full[st], ph, abort_flag, p.err))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ss(tD, smem_desc_sw128(a0 + st * kRTile + 32 * k, 16, 1024),
+                        smem_desc_sw128(b0 + st * kRB + 32 * k, 16, 1024), id_inter,
+                        (d_init || k > 0) ? 1u : 0u);
+          d_init = true;
+          mma_commit(&a_empty[st]);
+          mma_commit(&b_empty[st]);
+          intra(false);
+        }
+      }
+      if (ok) intra(true);
+      mma_commit(o_full);  // also orders every MMA before the final TMEM release
+      if (!ok) {
+        volatile int never = 0;
+        mbar_wait(o_full, 0, &never, p.err);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- epilogue: in-chunk Taylor scores, then normalisation
+    const int q4 = warp & 3;
+    const int row = 32 * q4 + lane;
+    const int tok = t0 + row;
+    const uint32_t tl = (uint32_t)(32 * q4) << 16;
+    bool ok = true;
+    for (int kb = 0; ok && kb < nkb; ++kb) {
+      if (!(ok = mbar_wait(s_full, kb & 1, abort_flag, p.err))) break;
+      tc_fence_after();
+      {
+        uint32_t v[kKB];
+#pragma unroll
+        for (int j = 0; j < kKB / 16; ++j)
+          tmem_ld16(tS + tl + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+        tmem_ld_wait();
+        const int key0 = c0 + kKB * kb;
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int j = 0; j < kKB / 2; ++j) {
+          const int ka = key0 + 2 * j, kc = ka + 1;
+          const float ta = (ka <= tok && ka < p.N) ? taylor4(__uint_as_float(v[2 * j]) * 0.125f) : 0.f;
+          const float tb =
+              (kc <= tok && kc < p.N) ? taylor4(__uint_as_float(v[2 * j + 1]) * 0.125f) : 0.f;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(ta, tb);
+          const float2 hf = __bfloat1622float2(h2);
+          hi[j] = *reinterpret_cast<const uint32_t *>(&h2);
+          lo[j] = pack_bf16x2(ta - hf.x, tb - hf.y);
+        }
+        store_tile_row(sP, (uint32_t)row, hi);
+        store_tile_row(sP + kRTile, (uint32_t)row, lo);
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && (ok = mbar_wait(o_full, 0, abort_flag, p.err))) {
+      tc_fence_after();
+      uint32_t v[kNP];
+#pragma unroll
+      for (int j = 0; j < kNP / 16; ++j)
+        tmem_ld16(tD + tl + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+      tmem_ld_wait();
+      if (tok < p.N) {
+        const float den = __uint_as_float(v[64]);
+        float4 *dst = reinterpret_cast<float4 *>(p.out + ((size_t)bh * p.N + tok) * 64);
+#pragma unroll
+        for (int n = 0; n < 16; ++n)
+          dst[n] = make_float4(__uint_as_float(v[4 * n]) / den, __uint_as_float(v[4 * n + 1]) / den,
+                               __uint_as_float(v[4 * n + 2]) / den,
+                               __uint_as_float(v[4 * n + 3]) / den);
+      }
+    }
+  } else if (warp >= 8 && inter) {
+    // ---------------- feature generators: phi(Q) tiles, one thread per token
+    const int gw = warp - 8;
+    const int half = gw >> 2;
+    const int row = lane + 32 * (gw & 3);
+    bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
+    const uint8_t *qrow = sQ + row * kRow;
+    for (int i = half; ok && i < p.n_tiles; i += 2) {
+      const int st = i % kRStages;
+      if (i >= kRStages && !(ok = mbar_wait(&a_empty[st], ((i / kRStages) - 1) & 1, abort_flag,
+                                            p.err)))
+        break;
+      const TileDesc td = p.tiles[i];
+      uint32_t out[32];
+      gen_tile(td, qrow, (uint32_t)(row & 7), p.W, out);
+      store_tile_row(sA + st * kRTile, (uint32_t)row, out);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[st]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+// ============================================================ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)ptr;
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor {d0 (contiguous), d1, d2}, box {64, box1, 1}, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+              uint32_t box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const cuuint32_t box[3] = {64, box1, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+GenWeights weights64() {
+  const double d = 64.0;
+  GenWeights W;
+  W.w3 = (float)(1.0 / std::sqrt(std::pow(d, 1.5)));
+  W.w3h = (float)(1.0 / std::sqrt(2.0 * std::pow(d, 1.5)));
+  W.w3s = (float)(1.0 / std::sqrt(6.0 * std::pow(d, 1.5)));
+  W.w2 = (float)(1.0 / std::sqrt(d));
+  W.w2h = (float)(1.0 / std::sqrt(2.0 * d));
+  W.w1 = (float)(1.0 / std::sqrt(std::sqrt(d)));
+  return W;
+}
+
+}  // namespace
+
+bool tc_supported(int dK, int dV, int P, bool bf16) {
+  return bf16 && dK == 64 && dV == 64 && P == 4;
+}
+
+int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, float *state,
+                      int B, int H, int N, const DeviceBasis *basis, int *err,
+                      cudaStream_t stream) {
+  const int BH = B * H;
+  const int n_tiles = basis->n_tiles;  // even, padded
+  const int m_pad = n_tiles * 64;
+  const int C = N <= 1024 ? ((N + 127) / 128) * 128 : 1024;
+  const int nsnap = (N + C - 1) / C - 1;
+  const size_t per_head = (size_t)nsnap * 65 * m_pad * 2;
+  const size_t budget = (size_t)4 << 30;
+  int G = BH;
+  if (per_head > 0) G = (int)std::max<size_t>(1, std::min<size_t>(BH, budget / per_head));
+  __nv_bfloat16 *snap = nullptr;
+  if (per_head > 0) {
+    int st = SATA_OK;
+    snap = (__nv_bfloat16 *)get_workspace(stream, per_head * G, &st);
+    if (!snap) return st;
+  }
+  CUtensorMap mK64, mV64, mQ, mS;
+  if (!make_map(&mK64, k, 64, N, BH, 64) || !make_map(&mV64, v, 64, N, BH, 64) ||
+      !make_map(&mQ, q, 64, N, BH, 128))
+    return SATA_ERR_CUDA;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(tc_chunk_states, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kUSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(tc_readout, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmem) !=
+            cudaSuccess)
+      return SATA_ERR_CUDA;
+    attr_done = true;
+  }
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+
+  const int n_mt = n_tiles / 2;
+  const int n_batches = (n_mt + kUF - 1) / kUF;
+  const GenWeights W = weights64();
+  for (int h0 = 0; h0 < BH; h0 += G) {
+    const int g = std::min(G, BH - h0);
+    if (nsnap > 0 &&
+        !make_map(&mS, snap, (uint64_t)m_pad, 65, (uint64_t)g * nsnap, kNP))
+      return SATA_ERR_CUDA;
+    UParams up;
+    up.tiles = reinterpret_cast<const TileDesc *>(basis->tile_desc);
+    up.row_of_slot = basis->tile_row;
+    up.W = W;
+    up.n_tiles = n_tiles;
+    up.N = N;
+    up.C = C;
+    up.nsnap = nsnap;
+    up.m = (int)basis->m;
+    up.m_pad = m_pad;
+    up.n_batches = n_batches;
+    up.n_items = g * n_batches;
+    up.head0 = h0;
+    up.snap = snap;
+    up.state = state;
+    up.err = err;
+    prof_kernel_begin(stream, K_TC_CHUNK_STATES);
+    tc_chunk_states<<<std::min(up.n_items, nsm), kThreads, kUSmem, stream>>>(mK64, mV64, up);
+    prof_kernel_end(stream);
+    RParams rp;
+    rp.tiles = up.tiles;
+    rp.W = W;
+    rp.n_tiles = n_tiles;
+    rp.N = N;
+    rp.C = C;
+    rp.nsnap = nsnap;
+    rp.head0 = h0;
+    rp.out = out;
+    rp.err = err;
+    if (nsnap == 0) mS = mQ;  // never read: no chunk has a predecessor
+    prof_kernel_begin(stream, K_TC_READOUT);
+    tc_readout<<<dim3((N + 127) / 128, g), kThreads, kRSmem, stream>>>(mQ, mK64, mV64, mS, rp);
+    prof_kernel_end(stream);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace sata

@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "sata_internal.h"
+#include "tile_order.h"
 
 namespace sata {
 namespace {
@@ -73,6 +74,28 @@ const DeviceBasis *get_device_basis(int dK, int P, int *status) {
                 cudaSuccess &&
             cudaMemcpy(db->w, w.data(), hb.m * sizeof(float), cudaMemcpyHostToDevice) ==
                 cudaSuccess;
+  if (ok && dK == 64 && P == 4) {
+    // tile order for the tensor-core path, padded to an even number of tiles
+    TileOrder to;
+    if (!build_tile_order(dK, &to)) {
+      free_basis(db);
+      *status = SATA_ERR_CUDA;
+      return nullptr;
+    }
+    if (to.n_tiles % 2) {
+      to.tiles.push_back({T_PAD, 0, 0, 0, 0, 0, 0, 0});
+      to.row_of_slot.insert(to.row_of_slot.end(), 64, -1);
+      to.n_tiles++;
+    }
+    db->n_tiles = to.n_tiles;
+    db->m_pad = (int64_t)to.n_tiles * 64;
+    ok = cudaMalloc(&db->tile_desc, to.tiles.size() * sizeof(TileDesc)) == cudaSuccess &&
+         cudaMalloc(&db->tile_row, to.row_of_slot.size() * sizeof(int32_t)) == cudaSuccess &&
+         cudaMemcpy(db->tile_desc, to.tiles.data(), to.tiles.size() * sizeof(TileDesc),
+                    cudaMemcpyHostToDevice) == cudaSuccess &&
+         cudaMemcpy(db->tile_row, to.row_of_slot.data(), to.row_of_slot.size() * sizeof(int32_t),
+                    cudaMemcpyHostToDevice) == cudaSuccess;
+  }
   if (!ok) {
     free_basis(db);
     *status = SATA_ERR_NOMEM;
@@ -229,7 +252,14 @@ extern "C" int sata_prefill(const void *q, const void *k, const void *v, float *
   const DeviceBasis *basis = get_device_basis(dK, P, &st);
   if (!basis) return st;
   prof_call_begin();
-  return launch_prefill_simt(q, k, v, out, state, B, H, N, dK, dV, P, dt == SATA_BF16, basis,
+  const bool bf16 = dt == SATA_BF16;
+  static const bool force_simt = getenv("SATA_FORCE_SIMT") && getenv("SATA_FORCE_SIMT")[0] == '1';
+  if (!force_simt && tc_supported(dK, dV, P, bf16) && basis->tile_desc) {
+    int *err = device_error_ptr();
+    if (!err) return SATA_ERR_NOMEM;
+    return launch_prefill_tc(q, k, v, out, state, B, H, N, basis, err, (cudaStream_t)stream);
+  }
+  return launch_prefill_simt(q, k, v, out, state, B, H, N, dK, dV, P, bf16, basis,
                              (cudaStream_t)stream);
 }
 

@@ -36,7 +36,7 @@ struct DeviceBasis {
   // Tensor-core tile order (dK in {32, 64}, P == 4); null when not built.
   int n_tiles = 0;              // 64-feature tiles
   int64_t m_pad = 0;            // n_tiles * 64
-  uint32_t *tile_desc = nullptr;  // [n_tiles] packed tile descriptors
+  void *tile_desc = nullptr;      // [n_tiles] TileDesc (tile_order.h)
   int32_t *tile_row = nullptr;    // [m_pad] lexicographic row of each padded feature (-1 = pad)
 };
 
@@ -55,6 +55,12 @@ int *device_error_ptr();
 int launch_prefill_simt(const void *q, const void *k, const void *v, float *out,
                         float *state, int B, int H, int N, int dK, int dV, int P,
                         bool bf16, const DeviceBasis *basis, cudaStream_t stream);
+
+// Tensor-core prefill (bf16, dK = dV = 64, P = 4); basis must carry the tile order.
+bool tc_supported(int dK, int dV, int P, bool bf16);
+int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, float *state,
+                      int B, int H, int N, const DeviceBasis *basis, int *err,
+                      cudaStream_t stream);
 
 int launch_decode(const void *q, const void *k, const void *v, float *state, float *out,
                   int B, int H, int dK, int dV, int P, bool bf16,

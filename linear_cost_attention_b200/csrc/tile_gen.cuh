@@ -1,0 +1,271 @@
+// Device-side generation of one 64-feature tile of the tile order
+// (tile_order.h) for one token, dK = 64.
+//
+// The token's bf16 row (64 elements) sits in shared memory as a 128-byte row
+// in the 128-byte-swizzled layout a TMA load produces: element i is in 16-byte
+// chunk i/8, stored at chunk position (i/8) ^ (row % 8).  The 64 outputs are
+// returned as 32 packed bf16x2 words in tile order.
+//
+// Arithmetic (feature = w_alpha * prod x): OUTER and BC tiles form the pair
+// product u = w * x_i * x_j in fp32, round it to bf16 and multiply by the
+// eight values of the third octet with packed bf16x2 multiplies (two
+// roundings); D and MISC tiles (21 of 749) form each product in fp32 and round
+// once.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <string.h>
+
+#include <utility>
+
+#include "tc_common.cuh"
+#include "tile_order.h"
+
+#ifndef SATA_HD
+#define SATA_HD __host__ __device__ __forceinline__
+#endif
+
+namespace sata {
+namespace tc {
+
+// Basis weights for dK = 64: 1/sqrt(alpha! * 64^(p/2)).
+struct GenWeights {
+  float w3, w3h;  // degree 3: alpha! = 1, 2  (64^-3/4 = 2^-4.5)
+  float w3s;      // degree 3: alpha! = 6
+  float w2, w2h;  // degree 2: alpha! = 1, 2
+  float w1;       // degree 1
+};
+
+SATA_HD float bits_f32(uint32_t b) {
+#ifdef __CUDA_ARCH__
+  return __uint_as_float(b);
+#else
+  float f;
+  memcpy(&f, &b, 4);
+  return f;
+#endif
+}
+
+SATA_HD float bf16_bits_to_f32(uint32_t bits16) { return bits_f32(bits16 << 16); }
+
+SATA_HD uint4 load_chunk(const uint8_t *row, uint32_t rsw, int c) {
+  return *reinterpret_cast<const uint4 *>(row + (((uint32_t)c ^ rsw) << 4));
+}
+
+SATA_HD void unpack8(uint4 r, float (&o)[8]) {
+  o[0] = bits_f32(r.x << 16);
+  o[1] = bits_f32(r.x & 0xffff0000u);
+  o[2] = bits_f32(r.y << 16);
+  o[3] = bits_f32(r.y & 0xffff0000u);
+  o[4] = bits_f32(r.z << 16);
+  o[5] = bits_f32(r.z & 0xffff0000u);
+  o[6] = bits_f32(r.w << 16);
+  o[7] = bits_f32(r.w & 0xffff0000u);
+}
+
+SATA_HD float load_elem(const uint8_t *row, uint32_t rsw, int i) {
+  const uint16_t b =
+      *reinterpret_cast<const uint16_t *>(row + ((((uint32_t)i >> 3) ^ rsw) << 4) + ((i & 7) << 1));
+  return bf16_bits_to_f32(b);
+}
+
+SATA_HD uint32_t bmul2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 x, y, z;
+  memcpy(&x, &a, 4);
+  memcpy(&y, &b, 4);
+  z = __hmul2(x, y);
+  uint32_t r;
+  memcpy(&r, &z, 4);
+  return r;
+}
+
+SATA_HD uint32_t splat_bf16(float u) {
+  __nv_bfloat162 v = __float2bfloat162_rn(u);
+  uint32_t r;
+  memcpy(&r, &v, 4);
+  return r;
+}
+
+SATA_HD uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  uint32_t r;
+  memcpy(&r, &v, 4);
+  return r;
+}
+
+// u * (8 values of chunk r) -> out[4*slot .. 4*slot+3]
+SATA_HD void scale_chunk(float u, uint4 r, uint32_t *out4) {
+  const uint32_t uu = splat_bf16(u);
+  out4[0] = bmul2(uu, r.x);
+  out4[1] = bmul2(uu, r.y);
+  out4[2] = bmul2(uu, r.z);
+  out4[3] = bmul2(uu, r.w);
+}
+
+SATA_HD void gen_outer(const TileDesc &td, const uint8_t *row, uint32_t rsw,
+                                          const GenWeights &W, uint32_t (&out)[32]) {
+  float ob[8];
+  unpack8(load_chunk(row, rsw, td.o0), ob);
+  const uint4 rc = load_chunk(row, rsw, td.o1);
+  const float s = (td.wsel == 0 ? W.w3 : W.w2) * (td.i1 < 64 ? load_elem(row, rsw, td.i1) : 1.f);
+#pragma unroll
+  for (int b = 0; b < 8; ++b) scale_chunk(s * ob[b], rc, &out[4 * b]);
+}
+
+// ---- BC: chunk CC of variant T
+template <int T, int CC>
+SATA_HD void bc_chunk(const float (&g0)[8], uint4 r0, const float (&g1)[8],
+                                         uint4 r1, const GenWeights &W, uint32_t (&out)[32]) {
+  constexpr int k = 8 * T + CC, blk = k / 36, p = k % 36;
+  constexpr int a = pair_a(p), b = pair_b(p);
+  const float w = (a == b) ? W.w3h : W.w3;
+  if (blk == 0)
+    scale_chunk(w * g0[a] * g0[b], r0, &out[4 * CC]);
+  else
+    scale_chunk(w * g1[a] * g1[b], r1, &out[4 * CC]);
+}
+
+template <int T, int... CC>
+SATA_HD void bc_variant(const float (&g0)[8], uint4 r0, const float (&g1)[8],
+                                           uint4 r1, const GenWeights &W, uint32_t (&out)[32],
+                                           std::integer_sequence<int, CC...>) {
+  (bc_chunk<T, CC>(g0, r0, g1, r1, W, out), ...);
+}
+
+template <int T>
+SATA_HD void gen_bc(const TileDesc &td, const uint8_t *row, uint32_t rsw,
+                                       const GenWeights &W, uint32_t (&out)[32]) {
+  constexpr bool need0 = 8 * T < 36, need1 = 8 * T + 7 >= 36;
+  float g0[8] = {0, 0, 0, 0, 0, 0, 0, 0}, g1[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
+  if (need0) {
+    unpack8(load_chunk(row, rsw, td.o0), g0);
+    r0 = load_chunk(row, rsw, td.o1);
+  }
+  if (need1) {
+    unpack8(load_chunk(row, rsw, td.o2), g1);
+    r1 = load_chunk(row, rsw, td.o3);
+  }
+  bc_variant<T>(g0, r0, g1, r1, W, out, std::make_integer_sequence<int, 8>{});
+}
+
+// ---- D: features 64*T + P of the concatenated in-octet triples
+template <int T, int P>
+SATA_HD float d_feature(const uint8_t *row, uint32_t rsw, const GenWeights &W) {
+  constexpr int f = 64 * T + P;
+  if constexpr (f >= 120 * 8) {
+    return 0.f;
+  } else {
+    constexpr int g = f / 120, r = f % 120;
+    constexpr int a = 8 * g + triple_at(r, 0), b = 8 * g + triple_at(r, 1),
+                  c = 8 * g + triple_at(r, 2);
+    constexpr int fa = fact3(a, b, c);
+    const float w = fa == 1 ? W.w3 : fa == 2 ? W.w3h : W.w3s;
+    return w * load_elem(row, rsw, a) * load_elem(row, rsw, b) * load_elem(row, rsw, c);
+  }
+}
+
+template <int T, int... Q>
+SATA_HD void d_variant(const uint8_t *row, uint32_t rsw, const GenWeights &W,
+                                          uint32_t (&out)[32], std::integer_sequence<int, Q...>) {
+  ((out[Q] = pack2(d_feature<T, 2 * Q>(row, rsw, W), d_feature<T, 2 * Q + 1>(row, rsw, W))),
+   ...);
+}
+
+// ---- MISC: in-octet pairs (degree 2), degree 1, degree 0, padding
+template <int T, int P>
+SATA_HD float misc_feature(const uint8_t *row, uint32_t rsw,
+                                              const GenWeights &W) {
+  constexpr int f = 64 * T + P;
+  constexpr int n2 = 36 * 8, n1 = 64;
+  if constexpr (f < n2) {
+    constexpr int g = f / 36, pr = f % 36;
+    constexpr int a = 8 * g + pair_a(pr), b = 8 * g + pair_b(pr);
+    return (a == b ? W.w2h : W.w2) * load_elem(row, rsw, a) * load_elem(row, rsw, b);
+  } else if constexpr (f < n2 + n1) {
+    return W.w1 * load_elem(row, rsw, f - n2);
+  } else if constexpr (f == n2 + n1) {
+    return 1.f;
+  } else {
+    return 0.f;
+  }
+}
+
+template <int T, int... Q>
+SATA_HD void misc_variant(const uint8_t *row, uint32_t rsw,
+                                             const GenWeights &W, uint32_t (&out)[32],
+                                             std::integer_sequence<int, Q...>) {
+  ((out[Q] = pack2(misc_feature<T, 2 * Q>(row, rsw, W),
+                         misc_feature<T, 2 * Q + 1>(row, rsw, W))),
+   ...);
+}
+
+// Generates tile td for the token whose swizzled row starts at `row`
+// (rsw = row index % 8 of that token inside its 8-row atom).
+SATA_HD void gen_tile(const TileDesc &td, const uint8_t *row, uint32_t rsw,
+                                         const GenWeights &W, uint32_t (&out)[32]) {
+  switch (td.type) {
+    case T_OUTER:
+      gen_outer(td, row, rsw, W, out);
+      return;
+    case T_BC:
+      switch (td.variant) {
+        case 0: gen_bc<0>(td, row, rsw, W, out); return;
+        case 1: gen_bc<1>(td, row, rsw, W, out); return;
+        case 2: gen_bc<2>(td, row, rsw, W, out); return;
+        case 3: gen_bc<3>(td, row, rsw, W, out); return;
+        case 4: gen_bc<4>(td, row, rsw, W, out); return;
+        case 5: gen_bc<5>(td, row, rsw, W, out); return;
+        case 6: gen_bc<6>(td, row, rsw, W, out); return;
+        case 7: gen_bc<7>(td, row, rsw, W, out); return;
+        default: gen_bc<8>(td, row, rsw, W, out); return;
+      }
+    case T_D: {
+      constexpr auto seq = std::make_integer_sequence<int, 32>{};
+      switch (td.variant) {
+        case 0: d_variant<0>(row, rsw, W, out, seq); return;
+        case 1: d_variant<1>(row, rsw, W, out, seq); return;
+        case 2: d_variant<2>(row, rsw, W, out, seq); return;
+        case 3: d_variant<3>(row, rsw, W, out, seq); return;
+        case 4: d_variant<4>(row, rsw, W, out, seq); return;
+        case 5: d_variant<5>(row, rsw, W, out, seq); return;
+        case 6: d_variant<6>(row, rsw, W, out, seq); return;
+        case 7: d_variant<7>(row, rsw, W, out, seq); return;
+        case 8: d_variant<8>(row, rsw, W, out, seq); return;
+        case 9: d_variant<9>(row, rsw, W, out, seq); return;
+        case 10: d_variant<10>(row, rsw, W, out, seq); return;
+        case 11: d_variant<11>(row, rsw, W, out, seq); return;
+        case 12: d_variant<12>(row, rsw, W, out, seq); return;
+        case 13: d_variant<13>(row, rsw, W, out, seq); return;
+        default: d_variant<14>(row, rsw, W, out, seq); return;
+      }
+    }
+    case T_MISC: {
+      constexpr auto seq = std::make_integer_sequence<int, 32>{};
+      switch (td.variant) {
+        case 0: misc_variant<0>(row, rsw, W, out, seq); return;
+        case 1: misc_variant<1>(row, rsw, W, out, seq); return;
+        case 2: misc_variant<2>(row, rsw, W, out, seq); return;
+        case 3: misc_variant<3>(row, rsw, W, out, seq); return;
+        case 4: misc_variant<4>(row, rsw, W, out, seq); return;
+        default: misc_variant<5>(row, rsw, W, out, seq); return;
+      }
+    }
+    default:
+#pragma unroll
+      for (int i = 0; i < 32; ++i) out[i] = 0u;
+      return;
+  }
+}
+
+// Stores the 64 generated features as row `r` of a 128-byte-swizzled tile.
+__device__ __forceinline__ void store_tile_row(uint8_t *tile, uint32_t r,
+                                               const uint32_t (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4 *>(tile + sw128_offset(r, (uint32_t)c)) =
+        make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+
+}  // namespace tc
+}  // namespace sata

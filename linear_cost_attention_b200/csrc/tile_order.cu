@@ -1,0 +1,138 @@
+// Host construction of the tensor-core tile order (see tile_order.h).
+#include <algorithm>
+#include <array>
+#include <map>
+
+#include "sata_internal.h"
+#include "tile_order.h"
+
+namespace sata {
+namespace {
+
+// key of a sorted tuple of degree deg (unused slots 0xff)
+uint32_t tuple_key(int deg, int i, int j, int l) {
+  return (uint32_t)deg | (uint32_t)(i & 0xff) << 8 | (uint32_t)(j & 0xff) << 16 |
+         (uint32_t)(l & 0xff) << 24;
+}
+
+struct Slot {
+  int deg;  // -1 = padding
+  int i, j, l;
+};
+
+Slot sorted3(int x, int y, int z) {
+  int v[3] = {x, y, z};
+  std::sort(v, v + 3);
+  return {3, v[0], v[1], v[2]};
+}
+Slot sorted2(int x, int y) { return {2, std::min(x, y), std::max(x, y), -1}; }
+
+}  // namespace
+
+bool build_tile_order(int dK, TileOrder *out) {
+  if (dK != 64) return false;
+  const int G = dK / 8;
+  HostBasis hb = build_host_basis(dK, 4);
+  std::map<uint32_t, int32_t> lex;
+  for (int64_t r = 0; r < hb.m; ++r) {
+    const int deg = hb.degree[r];
+    int ix[3] = {-1, -1, -1};
+    for (int s = 0; s < deg; ++s) ix[s] = hb.ix[3 * r + s];
+    lex[tuple_key(deg, ix[0], ix[1], ix[2])] = (int32_t)r;
+  }
+  std::vector<TileDesc> tiles;
+  std::vector<Slot> slots;
+  auto push = [&](TileDesc td, const std::array<Slot, 64> &s) {
+    tiles.push_back(td);
+    slots.insert(slots.end(), s.begin(), s.end());
+  };
+  std::array<Slot, 64> s;
+  // OUTER, degree 3: three distinct octets
+  for (int gi = 0; gi < G; ++gi)
+    for (int gj = gi + 1; gj < G; ++gj)
+      for (int gl = gj + 1; gl < G; ++gl)
+        for (int a = 0; a < 8; ++a) {
+          for (int b = 0; b < 8; ++b)
+            for (int c = 0; c < 8; ++c) s[8 * b + c] = sorted3(8 * gi + a, 8 * gj + b, 8 * gl + c);
+          push({T_OUTER, 0, (uint8_t)(8 * gi + a), (uint8_t)gj, (uint8_t)gl, 0, 0, 0}, s);
+        }
+  // BC: pairs of ordered octet pairs (g, g'), g != g'
+  std::vector<std::pair<int, int>> og;
+  for (int g = 0; g < G; ++g)
+    for (int h = 0; h < G; ++h)
+      if (h != g) og.push_back({g, h});
+  for (size_t bp = 0; bp + 1 < og.size(); bp += 2) {
+    const auto b0 = og[bp], b1 = og[bp + 1];
+    for (int t = 0; t < 9; ++t) {
+      for (int cc = 0; cc < 8; ++cc) {
+        const int k = 8 * t + cc, blk = k / 36, p = k % 36;
+        const int a = pair_a(p), b = pair_b(p);
+        const auto gg = blk ? b1 : b0;
+        for (int e = 0; e < 8; ++e)
+          s[8 * cc + e] = sorted3(8 * gg.first + a, 8 * gg.first + b, 8 * gg.second + e);
+      }
+      push({T_BC, (uint8_t)t, 0, (uint8_t)b0.first, (uint8_t)b0.second, (uint8_t)b1.first,
+            (uint8_t)b1.second, 0},
+           s);
+    }
+  }
+  // OUTER, degree 2: two distinct octets
+  for (int g = 0; g < G; ++g)
+    for (int h = g + 1; h < G; ++h) {
+      for (int b = 0; b < 8; ++b)
+        for (int c = 0; c < 8; ++c) s[8 * b + c] = sorted2(8 * g + b, 8 * h + c);
+      push({T_OUTER, 0, (uint8_t)dK, (uint8_t)g, (uint8_t)h, 0, 0, 1}, s);
+    }
+  // D: triples inside one octet
+  const int nD = (120 * G + 63) / 64;
+  for (int t = 0; t < nD; ++t) {
+    for (int p = 0; p < 64; ++p) {
+      const int f = 64 * t + p;
+      if (f < 120 * G) {
+        const int g = f / 120, r = f % 120;
+        s[p] = {3, 8 * g + triple_at(r, 0), 8 * g + triple_at(r, 1), 8 * g + triple_at(r, 2)};
+      } else {
+        s[p] = {-1, -1, -1, -1};
+      }
+    }
+    push({T_D, (uint8_t)t, 0, 0, 0, 0, 0, 0}, s);
+  }
+  // MISC: degree-2 pairs inside one octet, degree 1, degree 0, padding
+  const int nMisc = 36 * G + dK + 1;
+  const int nM = (nMisc + 63) / 64;
+  for (int t = 0; t < nM; ++t) {
+    for (int p = 0; p < 64; ++p) {
+      const int f = 64 * t + p;
+      if (f < 36 * G) {
+        const int g = f / 36, pr = f % 36;
+        s[p] = {2, 8 * g + pair_a(pr), 8 * g + pair_b(pr), -1};
+      } else if (f < 36 * G + dK) {
+        s[p] = {1, f - 36 * G, -1, -1};
+      } else if (f == 36 * G + dK) {
+        s[p] = {0, -1, -1, -1};
+      } else {
+        s[p] = {-1, -1, -1, -1};
+      }
+    }
+    push({T_MISC, (uint8_t)t, 0, 0, 0, 0, 0, 0}, s);
+  }
+  // coverage check: every basis row exactly once
+  std::vector<int> hits(hb.m, 0);
+  out->row_of_slot.assign(slots.size(), -1);
+  for (size_t k = 0; k < slots.size(); ++k) {
+    const Slot &sl = slots[k];
+    if (sl.deg < 0) continue;
+    auto it = lex.find(tuple_key(sl.deg, sl.i, sl.j, sl.l));
+    if (it == lex.end()) return false;
+    out->row_of_slot[k] = it->second;
+    hits[it->second]++;
+  }
+  for (int64_t r = 0; r < hb.m; ++r)
+    if (hits[r] != 1) return false;
+  out->dK = dK;
+  out->n_tiles = (int)tiles.size();
+  out->tiles = tiles;
+  return true;
+}
+
+}  // namespace sata

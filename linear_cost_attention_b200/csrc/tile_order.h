@@ -1,0 +1,80 @@
+// Tile order of the minimal basis for the tensor-core path (dK = 64, P = 4).
+//
+// The basis rows (sorted index tuples, "对称张量分解的核心洞察") are regrouped
+// into tiles of 64 features whose structure is fixed, so that one thread per
+// token can generate a tile with compile-time register indices.  Indices are
+// split into octets g = i / 8 (8 octets for dK = 64):
+//
+//  OUTER  x[i1] * x[8*ga + b] * x[8*gb + c], b, c = 0..7 (64 features):
+//         degree 3 with three distinct octets gi < gj < gl (i1 = 8*gi + a;
+//         56 octet triples x 8 values of a = 448 tiles), and degree 2 with
+//         two distinct octets (i1 absent; 28 tiles).
+//  BC     degree 3 with exactly two equal octets: a pair a <= b inside octet
+//         g times a full octet g' != g, 36 x 8 = 288 features per ordered
+//         (g, g'); two such blocks fill 9 tiles (252 tiles).
+//  D      degree 3 inside one octet: the 120 triples a <= b <= c of each
+//         octet, concatenated over the 8 octets (15 tiles).
+//  MISC   degree 2 inside one octet (36 pairs per octet), degree 1 (64),
+//         degree 0 (1), zero padding (6 tiles).
+// 749 tiles = 47936 slots for the 47905 rows; 31 slots are zero padding.  Per
+// feature, the weight is the basis weight 1/sqrt(alpha! dK^(p/2)) of its row.
+#pragma once
+
+#include <stdint.h>
+
+#include <vector>
+
+namespace sata {
+
+enum TileType : uint8_t { T_OUTER = 0, T_BC = 1, T_D = 2, T_MISC = 3, T_PAD = 4 };
+
+struct TileDesc {  // 8 bytes; read by the generator warps
+  uint8_t type, variant, i1, o0, o1, o2, o3, wsel;
+};
+
+// Index pairs a <= b and triples a <= b <= c inside one octet, lexicographic.
+__host__ __device__ constexpr int pair_a(int p) {
+  int n = 0;
+  for (int a = 0; a < 8; ++a)
+    for (int b = a; b < 8; ++b) {
+      if (n == p) return a;
+      ++n;
+    }
+  return 0;
+}
+__host__ __device__ constexpr int pair_b(int p) {
+  int n = 0;
+  for (int a = 0; a < 8; ++a)
+    for (int b = a; b < 8; ++b) {
+      if (n == p) return b;
+      ++n;
+    }
+  return 0;
+}
+__host__ __device__ constexpr int triple_at(int r, int which) {
+  int n = 0;
+  for (int a = 0; a < 8; ++a)
+    for (int b = a; b < 8; ++b)
+      for (int c = b; c < 8; ++c) {
+        if (n == r) return which == 0 ? a : which == 1 ? b : c;
+        ++n;
+      }
+  return 0;
+}
+// alpha! of a sorted triple / pair with equal-index runs
+__host__ __device__ constexpr int fact3(int a, int b, int c) {
+  return (a == b && b == c) ? 6 : (a == b || b == c) ? 2 : 1;
+}
+
+struct TileOrder {
+  int dK = 0;
+  int n_tiles = 0;
+  std::vector<TileDesc> tiles;
+  std::vector<int32_t> row_of_slot;  // [n_tiles*64] lexicographic basis row, -1 = padding
+};
+
+// Builds the tile order for dK = 64, P = 4 and checks that it covers every
+// basis row exactly once.  Returns false if the check fails.
+bool build_tile_order(int dK, TileOrder *out);
+
+}  // namespace sata

@@ -1,0 +1,90 @@
+// Host-only check of the tensor-core tile order and of its feature generator
+// (the device generator compiled for the host).  Built by
+// tests/test_tile_order_cpu.py with nvcc; needs no GPU.
+//   1. every basis row appears in exactly one tile slot;
+//   2. for random bf16 rows, every generated feature equals the basis weight
+//      times the product of its indexed entries, up to bf16 rounding.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <random>
+#include <vector>
+
+#include "../../linear_cost_attention_b200/csrc/sata_internal.h"
+#include "../../linear_cost_attention_b200/csrc/tile_gen.cuh"
+#include "../../linear_cost_attention_b200/csrc/tile_order.h"
+
+using namespace sata;
+
+int main() {
+  TileOrder to;
+  if (!build_tile_order(64, &to)) {
+    printf("FAIL build_tile_order\n");
+    return 1;
+  }
+  HostBasis hb = build_host_basis(64, 4);
+  printf("tiles %d slots %zu rows %lld\n", to.n_tiles, to.row_of_slot.size(), (long long)hb.m);
+  if (to.n_tiles != 749) {
+    printf("FAIL tile count\n");
+    return 1;
+  }
+  tc::GenWeights W;
+  W.w3 = (float)(1.0 / std::sqrt(512.0));
+  W.w3h = (float)(1.0 / std::sqrt(1024.0));
+  W.w3s = (float)(1.0 / std::sqrt(3072.0));
+  W.w2 = 0.125f;
+  W.w2h = (float)(1.0 / std::sqrt(128.0));
+  W.w1 = (float)(1.0 / std::sqrt(8.0));
+  std::mt19937 rng(1234);
+  std::normal_distribution<float> nd(0.f, 1.f);
+  double worst = 0;
+  long bad = 0;
+  for (int trial = 0; trial < 16; ++trial) {
+    // a token row in the 128-byte swizzled layout, at row index r (swizzle r % 8)
+    const uint32_t r = trial % 8;
+    float x[64];
+    uint16_t bits[64];
+    for (int i = 0; i < 64; ++i) {
+      __nv_bfloat16 b = __float2bfloat16_rn(trial == 15 ? (float)(i % 7) - 3.f : nd(rng));
+      x[i] = __bfloat162float(b);
+      memcpy(&bits[i], &b, 2);
+    }
+    alignas(16) uint8_t row[128];
+    for (int i = 0; i < 64; ++i) {
+      const int c = i / 8, e = i % 8;
+      memcpy(row + (((uint32_t)c ^ r) << 4) + 2 * e, &bits[i], 2);
+    }
+    for (int t = 0; t < to.n_tiles; ++t) {
+      uint32_t out[32];
+      tc::gen_tile(to.tiles[t], row, r, W, out);
+      for (int p = 0; p < 64; ++p) {
+        uint16_t h = (uint16_t)((out[p / 2] >> (16 * (p % 2))) & 0xffff);
+        __nv_bfloat16 hbv;
+        memcpy(&hbv, &h, 2);
+        const float got = __bfloat162float(hbv);
+        const int32_t row_id = to.row_of_slot[(size_t)t * 64 + p];
+        double ref = 0.0;
+        if (row_id >= 0) {
+          ref = hb.weight[row_id];
+          for (int s = 0; s < hb.degree[row_id]; ++s) ref *= x[hb.ix[3 * row_id + s]];
+        }
+        const double err = std::fabs(got - ref);
+        const double tol = 3 * std::ldexp(1.0, -8) * std::fabs(ref) + 1e-30;
+        if (row_id < 0 ? got != 0.f : err > tol) {
+          if (bad < 10)
+            printf("mismatch tile %d type %d var %d slot %d row %d got %g ref %g\n", t,
+                   to.tiles[t].type, to.tiles[t].variant, p, row_id, got, ref);
+          ++bad;
+        }
+        if (ref != 0) worst = std::fmax(worst, err / std::fabs(ref));
+      }
+    }
+  }
+  printf("worst relative %.3e bad %ld\n", worst, bad);
+  if (bad) {
+    printf("FAIL\n");
+    return 1;
+  }
+  printf("OK\n");
+  return 0;
+}

@@ -93,6 +93,21 @@ def test_edge_shapes(B, H, N, dK, dV, P, dt):
     check_prefill(q, k, v, P, TOL[dt])
 
 
+@pytest.mark.parametrize("B,H,N", [
+    (1, 1, 1),        # one token
+    (1, 2, 100),      # ragged, one partial key block
+    (1, 1, 128),      # exactly one block, no snapshot
+    (2, 1, 1024),     # one full chunk
+    (1, 2, 1152),     # one snapshot + a block of the next chunk
+    (1, 1, 2500),     # two snapshots, ragged tail
+    (1, 3, 4096),     # three snapshots, several items per head
+])
+def test_tensor_core_prefill_shapes(B, H, N):
+    # bf16, dK = dV = 64, P = 4: the tcgen05 path
+    q, k, v = make_qkv(B, H, N, 64, 64, seed=7 * N + H, dtype="bf16")
+    check_prefill(q, k, v, 4, TOL["bf16"])
+
+
 def test_invalid_call_raises():
     q = torch.zeros(1, 1, 4, 8, device="cuda")
     with pytest.raises(sata.SataError):
