@@ -63,44 +63,62 @@ __device__ __forceinline__ void fill_ones(uint8_t *blk, int rows) {
 }
 
 // ============================================================ chunk states
-constexpr int kUF = 4;                               // 128-row state tiles per item
-constexpr int kUT = 64;                              // tokens per step
-constexpr uint32_t kUTileBytes = kUT * kRow;         // 64 rows x 64 tokens: 8 KiB
-constexpr uint32_t kUAStage = 2 * kUF * kUTileBytes;  // 64 KiB
-constexpr uint32_t kUKV = kUT * kRow;                // 8 KiB
-constexpr uint32_t kUOffA = 0, kUOffK = 2 * kUAStage, kUOffV = kUOffK + 2 * kUKV,
-                   kUOffOnes = kUOffV + 2 * kUKV, kUOffBar = kUOffOnes + kUKV;
+// One CTA per (head, kUF x 128 basis rows).  Thread = basis row = TMEM lane:
+// each generator thread forms its row's unweighted monomial x_i x_j x_l for 64
+// tokens from the transposed keys (rows of K^T; index 64 is a row of ones that
+// is zero past the sequence end) and stores them with tcgen05.st straight into
+// the A operand in TMEM (basis rows x tokens, two tokens per column).  The MMA
+// accumulates S' += m(K)^T [V, 1]; the basis weights are applied when S' leaves
+// TMEM: state = w S', snapshot = w^2 S' (the readout then multiplies by the
+// unweighted m(q): sum_a w_a m_a(q) w_a S'_a = phi(q) . S).
+constexpr int kUF = 3;          // 128-row state tiles per item
+constexpr int kUT = 64;         // tokens per step
+constexpr int kUAS = 2;         // A stages (TMEM)
+constexpr int kUKS = 6;         // K^T / V stages (shared memory)
+constexpr int kUGenWarps = 4 * kUF;
+constexpr int kUThreads = 32 * (2 + kUGenWarps);
+constexpr int kMaxTiles = 768;  // tile table capacity in smem (readout)
+constexpr uint32_t kUColA = 256;               // TMEM: D at f*80, A from column 256
+constexpr uint32_t kUTmemCols = 512;
+constexpr uint32_t kUKT = 9 * 1024;            // 65 rows x 128 B, padded to 9 KiB
+constexpr uint32_t kUV = kUT * kRow;           // 8 KiB
+constexpr uint32_t kUOffKT = 0, kUOffV = kUOffKT + kUKS * kUKT, kUOffOnes = kUOffV + kUKS * kUV,
+                   kUOffBar = kUOffOnes + kUV;
 constexpr uint32_t kUSmem = kUOffBar + 256 + 1024;
+static_assert(kUColA + kUAS * kUF * 32 <= 512 && kUF * kNP <= kUColA, "TMEM budget");
 
 struct UParams {
-  const TileDesc *tiles;
+  const uint32_t *slot_idx;  // [m_pad] i | j << 8 | l << 16 (64 = the ones row)
+  const float *slot_w;       // [m_pad] basis weight (0 on padding)
   const int32_t *row_of_slot;
-  GenWeights W;
-  int n_tiles;  // even
+  int n_mt;                  // 128-row tiles (m_pad / 128)
   int N, C, nsnap, m, m_pad, n_batches, n_items, head0;
   __nv_bfloat16 *snap;  // [G][nsnap][65][m_pad]
   float *state;         // [BH][m][65]
   int *err;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
-    tc_chunk_states(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+__global__ void __launch_bounds__(kUThreads, 1)
+    tc_chunk_states(const __grid_constant__ CUtensorMap tmKT, const __grid_constant__ CUtensorMap tmV,
                     const UParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sA = smem + kUOffA, *sK = smem + kUOffK, *sV = smem + kUOffV, *sOnes = smem + kUOffOnes;
+  uint8_t *sKT = smem + kUOffKT, *sV = smem + kUOffV, *sOnes = smem + kUOffOnes;
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kUOffBar);
-  uint64_t *kv_full = bar, *kv_empty = bar + 2, *a_full = bar + 4, *a_empty = bar + 6,
-           *snap_full = bar + 8, *snap_done = bar + 9, *drain = bar + 13;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 14);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 15);
+  uint64_t *kv_full = bar, *kv_empty = bar + kUKS, *a_full = bar + 2 * kUKS,
+           *a_empty = a_full + kUAS, *snap_full = a_empty + kUAS, *snap_done = snap_full + 1,
+           *drain = snap_done + kUF;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(drain + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kUKS; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1 + 8);
-      mbar_init(&a_full[s], 8);
+      mbar_init(&kv_empty[s], 1 + kUGenWarps);
+    }
+    for (int s = 0; s < kUAS; ++s) {
+      mbar_init(&a_full[s], kUGenWarps);
       mbar_init(&a_empty[s], 1);
     }
     mbar_init(snap_full, 1);
@@ -111,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   fill_ones(sOnes, kUT);
   fence_proxy_async_smem();
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == 1) tmem_alloc(tmem_slot, kUTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -119,50 +137,50 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int nsub = (p.N + kUT - 1) / kUT;
   const int sub_per_chunk = p.C / kUT;
-  const int n_mt = p.n_tiles / 2;
+  auto is_event = [&](int s) {
+    return s == nsub - 1 || (((s + 1) % sub_per_chunk == 0) && (s + 1 < nsub));
+  };
 
   if (warp == 0) {
-    // ---------------- TMA producer: K and V rows of 64 tokens
+    // ---------------- TMA producer: K^T (65 rows x 64 tokens) and V (64 x 64)
     if (lane == 0) {
-      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmKT);
       prefetch_tensormap(&tmV);
       uint32_t it = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int bh = p.head0 + item / p.n_batches;
+        const int hb = item / p.n_batches, bh = p.head0 + hb;
         for (int s = 0; s < nsub; ++s, ++it) {
-          const int st = it & 1;
-          if (it >= 2 && !(ok = mbar_wait(&kv_empty[st], ((it >> 1) - 1) & 1, abort_flag, p.err)))
+          const int st = it % kUKS;
+          if (it >= kUKS &&
+              !(ok = mbar_wait(&kv_empty[st], ((it / kUKS) - 1) & 1, abort_flag, p.err)))
             break;
-          mbar_arrive_expect_tx(&kv_full[st], 2 * kUKV);
-          tma_load_3d(sK + st * kUKV, &tmK, &kv_full[st], 0, s * kUT, bh);
-          tma_load_3d(sV + st * kUKV, &tmV, &kv_full[st], 0, s * kUT, bh);
+          mbar_arrive_expect_tx(&kv_full[st], 65 * kRow + kUV);
+          tma_load_3d(sKT + st * kUKT, &tmKT, &kv_full[st], s * kUT, 0, hb);
+          tma_load_3d(sV + st * kUV, &tmV, &kv_full[st], 0, s * kUT, bh);
         }
       }
-      // let the loads already issued land before the CTA can exit
-      for (uint32_t j = it > 2 ? it - 2 : 0; j < it; ++j) {
+      for (uint32_t j = it > kUKS ? it - kUKS : 0; j < it; ++j) {
         volatile int never = 0;
-        mbar_wait(&kv_full[j & 1], (j >> 1) & 1, &never, p.err);
+        mbar_wait(&kv_full[j % kUKS], (j / kUKS) & 1, &never, p.err);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, kNP, true, true);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kNP, false, true);
       uint32_t it = 0, events = 0;
-      bool after_event = false;  // the epilogue must release each tile first
+      bool after_event = false;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const int batch = item % p.n_batches;
-        const int nmt = min(kUF, n_mt - batch * kUF);
+        const int nmt = min(kUF, p.n_mt - batch * kUF);
         for (int s = 0; ok && s < nsub; ++s, ++it) {
-          const int st = it & 1;
-          const uint32_t ph = (it >> 1) & 1;
-          if (!(ok = mbar_wait(&kv_full[st], ph, abort_flag, p.err))) break;
-          if (!(ok = mbar_wait(&a_full[st], ph, abort_flag, p.err))) break;
+          const int ks = it % kUKS, as = it % kUAS;
+          if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&a_full[as], (it / kUAS) & 1, abort_flag, p.err))) break;
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + st * kUAStage);
-          const uint32_t v0 = smem_u32(sV + st * kUKV);
+          const uint32_t v0 = smem_u32(sV + ks * kUV);
           const uint32_t lbo_b = smem_u32(sOnes) - v0;
           for (int f = 0; f < kUF; ++f) {
             // every tile's barrier is waited once per event, in order, so no
@@ -172,135 +190,165 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_after();
             }
             if (f >= nmt) continue;
+            const uint32_t a0 = tmem + kUColA + (as * kUF + f) * 32;
 #pragma unroll
             for (int k = 0; k < kUT / 16; ++k) {
-              const uint64_t ad = smem_desc_sw128(a0 + 2 * f * kUTileBytes + k * 2048,
-                                                  kUTileBytes, 1024);
               const uint64_t bd = smem_desc_sw128(v0 + k * 2048, lbo_b, 1024);
-              mma_bf16_ss(tmem + f * kNP, ad, bd, idesc, (s > 0 || k > 0) ? 1u : 0u);
+              mma_bf16_ts(tmem + f * kNP, a0 + 8 * k, bd, idesc, (s > 0 || k > 0) ? 1u : 0u);
             }
           }
           if (!ok) break;
           after_event = false;
-          mma_commit(&a_empty[st]);
-          mma_commit(&kv_empty[st]);
-          const bool boundary = ((s + 1) % sub_per_chunk == 0) && (s + 1 < nsub);
-          if (boundary || s == nsub - 1) {
+          mma_commit(&a_empty[as]);
+          mma_commit(&kv_empty[ks]);
+          if (is_event(s)) {
             mma_commit(snap_full);
             ++events;
             after_event = true;
           }
         }
       }
-      // every MMA issued so far completes before the TMEM is released
       mma_commit(drain);
       volatile int never = 0;
       mbar_wait(drain, 0, &never, p.err);
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ---------------- epilogue: snapshots and final state
-    const int q4 = warp & 3;
-    const int row = 32 * q4 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
-    uint32_t events = 0;
+  } else {
+    // ---------------- generators (one thread per basis row) and epilogue
+    const int g = warp - 2;
+    const int f = g >> 2;               // state tile of this warp
+    const int q4 = warp & 3;            // TMEM lane quarter
+    const int row = 32 * q4 + lane;     // basis row inside the tile
+    const uint32_t tl = (uint32_t)(32 * q4) << 16;
+    uint32_t it = 0, events = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
       const int hb = item / p.n_batches, batch = item % p.n_batches;
-      const int nmt = min(kUF, n_mt - batch * kUF);
-      for (int s = 0; s < nsub; ++s) {
-        const bool boundary = ((s + 1) % sub_per_chunk == 0) && (s + 1 < nsub);
-        if (!boundary && s != nsub - 1) continue;
-        if (!(ok = mbar_wait(snap_full, events & 1, abort_flag, p.err))) break;
+      const int mt = batch * kUF + f;
+      const bool live = mt < p.n_mt;
+      const int slot = mt * 128 + row;
+      uint32_t ix = 0x404040u;  // three "ones" rows
+      float w = 0.f;
+      if (live) {
+        ix = p.slot_idx[slot];
+        w = p.slot_w[slot];
+      }
+      const uint32_t ri = (ix & 0xff) * kRow, rj = ((ix >> 8) & 0xff) * kRow,
+                     rl = ((ix >> 16) & 0xff) * kRow;
+      const uint32_t si = (ix & 7), sj = ((ix >> 8) & 7), sl = ((ix >> 16) & 7);
+      auto epilogue = [&](int s) {
+        // S' of this tile for this lane quarter -> snapshot (w^2 S') or state (w S')
+        if (!(ok = mbar_wait(snap_full, events & 1, abort_flag, p.err))) return;
         ++events;
         tc_fence_after();
-        for (int f = 0; f < kUF; ++f) {
-          uint32_t v[kNP];
-          if (f < nmt) {
-#pragma unroll
-            for (int j = 0; j < kNP / 16; ++j)
-              tmem_ld16(tl + f * kNP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+        // 16 columns at a time (65 used of the 80): load, scale, store
+        const bool boundary = s != nsub - 1;
+        const int c = boundary ? (s + 1) / sub_per_chunk - 1 : 0;
+        const int r = (live && !boundary) ? p.row_of_slot[slot] : -1;
+        __nv_bfloat16 *sdst = p.snap + ((size_t)(hb * p.nsnap + c) * 65) * p.m_pad + slot;
+        float *tdst = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * 65;
+        const float scale = boundary ? w * w : w;
+#pragma unroll 1
+        for (int j = 0; j < 5; ++j) {
+          uint32_t v[16];
+          if (live) {
+            tmem_ld16(tmem + tl + f * kNP + 16 * j, v);
             tmem_ld_wait();
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&snap_done[f]);
-          if (f >= nmt) continue;
-          const int slot = (batch * kUF + f) * 128 + row;
+          if (j == 4) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&snap_done[f]);
+          }
+          if (!live) continue;
+          const int nmax = j == 4 ? 1 : 16;  // column 64 is the last one used
           if (boundary) {
-            const int c = (s + 1) / sub_per_chunk - 1;
-            __nv_bfloat16 *dst =
-                p.snap + ((size_t)(hb * p.nsnap + c) * 65) * p.m_pad + slot;
 #pragma unroll
-            for (int n = 0; n < 65; ++n)
-              dst[(size_t)n * p.m_pad] = __float2bfloat16_rn(__uint_as_float(v[n]));
-          } else {
-            const int r = p.row_of_slot[slot];
-            if (r >= 0) {
-              float *dst = p.state + ((size_t)(p.head0 + hb) * p.m + r) * 65;
+            for (int n = 0; n < 16; ++n)
+              if (n < nmax)
+                sdst[(size_t)(16 * j + n) * p.m_pad] =
+                    __float2bfloat16_rn(scale * __uint_as_float(v[n]));
+          } else if (r >= 0) {
 #pragma unroll
-              for (int n = 0; n < 65; ++n) dst[n] = __uint_as_float(v[n]);
-            }
+            for (int n = 0; n < 16; ++n)
+              if (n < nmax) tdst[16 * j + n] = scale * __uint_as_float(v[n]);
           }
         }
-      }
-    }
-  } else if (warp >= 8) {
-    // ---------------- feature generators: phi(K)^T tiles, one thread per token
-    const int gw = warp - 8;
-    const int t = lane + 32 * (gw & 1);
-    const int fq = gw >> 1;  // feature tiles fq and fq + 4 of the item
-    uint32_t it = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int batch = item % p.n_batches;
-      const int tile0 = batch * 2 * kUF;
-      for (int s = 0; s < nsub; ++s, ++it) {
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        if (!(ok = mbar_wait(&kv_full[st], ph, abort_flag, p.err))) break;
-        if (it >= 2 && !(ok = mbar_wait(&a_empty[st], ph ^ 1, abort_flag, p.err))) break;
-        const uint8_t *krow = sK + st * kUKV + t * kRow;
-        const bool valid = s * kUT + t < p.N;
-#pragma unroll 1
-        for (int j = fq; j < 2 * kUF; j += 4) {
-          const int ft = tile0 + j;
-          uint32_t out[32];
-          if (valid && ft < p.n_tiles) {
-            const TileDesc td = p.tiles[ft];
-            gen_tile(td, krow, (uint32_t)(t & 7), p.W, out);
-          } else {
+      };
+      for (int s = 0; ok && s < nsub; ++s, ++it) {
+        const int ks = it % kUKS, as = it % kUAS;
+        if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err))) break;
+        if (it >= kUAS &&
+            !(ok = mbar_wait(&a_empty[as], ((it / kUAS) - 1) & 1, abort_flag, p.err)))
+          break;
+        const uint8_t *kt = sKT + ks * kUKT;
+        uint32_t out[32];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) out[q] = 0u;
-          }
-          store_tile_row(sA + st * kUAStage + j * kUTileBytes, (uint32_t)t, out);
+        for (int c = 0; c < 8; ++c) {
+          const uint4 xi = *reinterpret_cast<const uint4 *>(kt + ri + (((uint32_t)c ^ si) << 4));
+          const uint4 xj = *reinterpret_cast<const uint4 *>(kt + rj + (((uint32_t)c ^ sj) << 4));
+          const uint4 xl = *reinterpret_cast<const uint4 *>(kt + rl + (((uint32_t)c ^ sl) << 4));
+          out[4 * c + 0] = bmul2(bmul2(xi.x, xj.x), xl.x);
+          out[4 * c + 1] = bmul2(bmul2(xi.y, xj.y), xl.y);
+          out[4 * c + 2] = bmul2(bmul2(xi.z, xj.z), xl.z);
+          out[4 * c + 3] = bmul2(bmul2(xi.w, xj.w), xl.w);
         }
-        fence_proxy_async_smem();
+        tmem_st32(tmem + tl + kUColA + (as * kUF + f) * 32, out);
+        tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&a_full[st]);
-          mbar_arrive(&kv_empty[st]);
+          mbar_arrive(&a_full[as]);
+          mbar_arrive(&kv_empty[ks]);
         }
+        // the previous step's snapshot, after this step's operand is handed over
+        if (s > 0 && is_event(s - 1)) epilogue(s - 1);
       }
+      if (ok && is_event(nsub - 1)) epilogue(nsub - 1);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 1) tmem_dealloc(tmem, kUTmemCols);
+}
+
+// K [BH, N, 64] -> K^T [BH, 65, Npad]: rows 0..63 the transposed keys, row 64
+// ones for t < N, zeros on the padding.
+__global__ void __launch_bounds__(256) tc_transpose_k(const __nv_bfloat16 *__restrict__ k,
+                                                      __nv_bfloat16 *__restrict__ kt, int N,
+                                                      int Npad, int head0) {
+  __shared__ __nv_bfloat16 tile[64][66];
+  const int t0 = blockIdx.x * 64;
+  const size_t bh = (size_t)head0 + blockIdx.y;
+  for (int e = threadIdx.x; e < 64 * 64; e += 256) {
+    const int t = e >> 6, d = e & 63;
+    tile[t][d] = (t0 + t < N) ? k[(bh * N + t0 + t) * 64 + d] : __float2bfloat16_rn(0.f);
+  }
+  __syncthreads();
+  __nv_bfloat16 *dst = kt + (size_t)blockIdx.y * 65 * Npad;
+  for (int e = threadIdx.x; e < 65 * 64; e += 256) {
+    const int d = e >> 6, t = e & 63;
+    dst[(size_t)d * Npad + t0 + t] =
+        d < 64 ? tile[t][d] : __float2bfloat16_rn(t0 + t < N ? 1.f : 0.f);
+  }
 }
 
 // ============================================================ readout
-constexpr int kRStages = 4;
+constexpr int kRStages = 10;             // phi(Q) stages, in TMEM (32 columns each)
+constexpr int kRBS = 12;                 // snapshot-tile stages (cover TMA latency)
 constexpr int kKB = 64;                  // keys per in-chunk block
 constexpr uint32_t kRTile = 128 * kRow;  // 128 tokens x 64 features: 16 KiB
 constexpr uint32_t kRB = kNP * kRow;     // 80 x 64 snapshot tile: 10 KiB
 constexpr uint32_t kRKV = kKB * kRow;    // 64 keys x 64: 8 KiB
-constexpr uint32_t kROffQ = 0, kROffA = kROffQ + kRTile, kROffB = kROffA + kRStages * kRTile,
-                   kROffK = kROffB + kRStages * kRB, kROffV = kROffK + kRKV,
+constexpr uint32_t kRColS = 96, kRColA = 160;  // TMEM: D 0..79, scores 96..159, A stages
+constexpr uint32_t kRTmemCols = 512;
+static_assert(kRColA + 32 * kRStages <= kRTmemCols, "TMEM budget");
+constexpr uint32_t kROffQ = 0, kROffB = kROffQ + kRTile,
+                   kROffK = kROffB + kRBS * kRB, kROffV = kROffK + kRKV,
                    kROffOnes = kROffV + kRKV, kROffP = kROffOnes + kRKV,
-                   kROffBar = kROffP + 2 * kRTile;
-constexpr uint32_t kRSmem = kROffBar + 256 + 1024;
+                   kROffTiles = kROffP + 2 * kRTile, kROffBar = kROffTiles + kMaxTiles * 8;
+constexpr uint32_t kRSmem = kROffBar + 512 + 1024;  // 50 barriers + TMEM slot + flag
 
 struct RParams {
   const TileDesc *tiles;
@@ -321,14 +369,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                const RParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sQ = smem + kROffQ, *sA = smem + kROffA, *sB = smem + kROffB, *sK = smem + kROffK,
+  uint8_t *sQ = smem + kROffQ, *sB = smem + kROffB, *sK = smem + kROffK,
           *sV = smem + kROffV, *sOnes = smem + kROffOnes, *sP = smem + kROffP;
+  TileDesc *sTiles = reinterpret_cast<TileDesc *>(smem + kROffTiles);
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kROffBar);
   uint64_t *q_full = bar, *kv_full = bar + 1, *kv_empty = bar + 2, *s_full = bar + 3,
-           *p_full = bar + 4, *o_full = bar + 5, *a_full = bar + 6, *a_empty = bar + 10,
-           *b_full = bar + 14, *b_empty = bar + 18;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 22);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 23);
+           *p_full = bar + 4, *o_full = bar + 5, *a_full = bar + 6, *a_empty = a_full + kRStages,
+           *b_full = a_empty + kRStages, *b_empty = b_full + kRBS;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(b_empty + kRBS);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(b_empty + kRBS + 1);
+  static_assert((6 + 2 * kRStages + 2 * kRBS + 2) * 8 <= 512, "barrier region");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * 128;
@@ -339,6 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nkb = (t0 - c0) / kKB + 128 / kKB;  // key blocks from the chunk start through t0+127
   const bool inter = chunk > 0;
 
+  if (inter)
+    for (int i = threadIdx.x; i < p.n_tiles; i += kThreads) sTiles[i] = p.tiles[i];
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(kv_full, 1);
@@ -349,6 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kRStages; ++s) {
       mbar_init(&a_full[s], 4);
       mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < kRBS; ++s) {
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], 1);
     }
@@ -357,12 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   fill_ones(sOnes, kKB);
   fence_proxy_async_smem();
-  if (warp == 1) tmem_alloc(tmem_slot, 256);
+  if (warp == 1) tmem_alloc(tmem_slot, kRTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tD = tmem, tS = tmem + 128;
+  const uint32_t tD = tmem, tS = tmem + kRColS;
 
   if (warp == 0) {
     // ---------------- TMA producer: snapshot tiles S_(c-1)[80 x 64 rows]
@@ -370,16 +424,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tmS);
       int i = 0;
       for (; i < p.n_tiles; ++i) {
-        const int st = i % kRStages;
-        if (i >= kRStages &&
-            !mbar_wait(&b_empty[st], ((i / kRStages) - 1) & 1, abort_flag, p.err))
+        const int st = i % kRBS;
+        if (i >= kRBS && !mbar_wait(&b_empty[st], ((i / kRBS) - 1) & 1, abort_flag, p.err))
           break;
         mbar_arrive_expect_tx(&b_full[st], kRB);
         tma_load_3d(sB + st * kRB, &tmS, &b_full[st], 64 * i, 0, hrel * p.nsnap + chunk - 1);
       }
-      for (int j = max(0, i - kRStages); j < i; ++j) {
+      for (int j = max(0, i - kRBS); j < i; ++j) {
         volatile int never = 0;
-        mbar_wait(&b_full[j % kRStages], (j / kRStages) & 1, &never, p.err);
+        mbar_wait(&b_full[j % kRBS], (j / kRBS) & 1, &never, p.err);
       }
     }
   } else if (warp == 2) {
@@ -418,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kb_qk == kb_pv) {  // next: scores of block kb_qk
             if (block) {
               if (!(ok = mbar_wait(kv_full, kb_qk & 1, abort_flag, p.err))) return;
-            } else if (!mbar_try_wait(kv_full, kb_qk & 1)) {
+            } else if (!mbar_test_wait(kv_full, kb_qk & 1)) {
               return;
             }
             tc_fence_after();
@@ -431,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {  // next: P [V, 1] of block kb_pv
             if (block) {
               if (!(ok = mbar_wait(p_full, kb_pv & 1, abort_flag, p.err))) return;
-            } else if (!mbar_try_wait(p_full, kb_pv & 1)) {
+            } else if (!mbar_test_wait(p_full, kb_pv & 1)) {
               return;
             }
             tc_fence_after();
@@ -450,21 +503,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       if (ok) intra(false);
       if (ok && inter) {
-        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+        const uint32_t b0 = smem_u32(sB);
         for (int i = 0; i < p.n_tiles; ++i) {
-          const int st = i % kRStages;
-          const uint32_t ph = (i / kRStages) & 1;
-          if (!(ok = mbar_wait(&a_full[st], ph, abort_flag, p.err))) break;
-          if (!(ok = mbar_wait(&b_full[st], ph, abort_flag, p.err))) break;
+          const int st = i % kRStages, bs = i % kRBS;
+          if (!(ok = mbar_wait(&a_full[st], (i / kRStages) & 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&b_full[bs], (i / kRBS) & 1, abort_flag, p.err))) break;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(tD, smem_desc_sw128(a0 + st * kRTile + 32 * k, 16, 1024),
-                        smem_desc_sw128(b0 + st * kRB + 32 * k, 16, 1024), id_inter,
+            mma_bf16_ts(tD, tmem + kRColA + st * 32 + 8 * k,
+                        smem_desc_sw128(b0 + bs * kRB + 32 * k, 16, 1024), id_inter,
                         (d_init || k > 0) ? 1u : 0u);
           d_init = true;
           mma_commit(&a_empty[st]);
-          mma_commit(&b_empty[st]);
+          mma_commit(&b_empty[bs]);
           intra(false);
         }
       }
@@ -541,11 +593,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i >= kRStages && !(ok = mbar_wait(&a_empty[st], ((i / kRStages) - 1) & 1, abort_flag,
                                             p.err)))
         break;
-      const TileDesc td = p.tiles[i];
+      const TileDesc td = sTiles[i];
       uint32_t out[32];
       gen_tile(td, qrow, (uint32_t)(row & 7), p.W, out);
-      store_tile_row(sA + st * kRTile, (uint32_t)row, out);
-      fence_proxy_async_smem();
+      // this thread's token is TMEM lane `row`; the tile's 64 features are 32
+      // packed columns of stage st
+      tmem_st32(tmem + ((uint32_t)(32 * (gw & 3)) << 16) + kRColA + st * 32, out);
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&a_full[st]);
     }
@@ -554,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, kRTmemCols);
 }
 
 // ============================================================ host side
@@ -590,17 +645,6 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-GenWeights weights64() {
-  const double d = 64.0;
-  GenWeights W;
-  W.w3 = (float)(1.0 / std::sqrt(std::pow(d, 1.5)));
-  W.w3h = (float)(1.0 / std::sqrt(2.0 * std::pow(d, 1.5)));
-  W.w3s = (float)(1.0 / std::sqrt(6.0 * std::pow(d, 1.5)));
-  W.w2 = (float)(1.0 / std::sqrt(d));
-  W.w2h = (float)(1.0 / std::sqrt(2.0 * d));
-  W.w1 = (float)(1.0 / std::sqrt(std::sqrt(d)));
-  return W;
-}
 
 }  // namespace
 
@@ -613,21 +657,24 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
                       cudaStream_t stream) {
   const int BH = B * H;
   const int n_tiles = basis->n_tiles;  // even, padded
+  if (n_tiles > kMaxTiles) return SATA_ERR_UNSUPPORTED;
   const int m_pad = n_tiles * 64;
   const int C = N <= 1024 ? ((N + 127) / 128) * 128 : 1024;
   const int nsnap = (N + C - 1) / C - 1;
-  const size_t per_head = (size_t)nsnap * 65 * m_pad * 2;
+  const int Npad = ((N + kUT - 1) / kUT) * kUT;
+  const size_t snap_head = (size_t)nsnap * 65 * m_pad * 2;
+  const size_t kt_head = (size_t)65 * Npad * 2;
+  const size_t per_head = snap_head + kt_head;
   const size_t budget = (size_t)4 << 30;
-  int G = BH;
-  if (per_head > 0) G = (int)std::max<size_t>(1, std::min<size_t>(BH, budget / per_head));
-  __nv_bfloat16 *snap = nullptr;
-  if (per_head > 0) {
-    int st = SATA_OK;
-    snap = (__nv_bfloat16 *)get_workspace(stream, per_head * G, &st);
-    if (!snap) return st;
-  }
-  CUtensorMap mK64, mV64, mQ, mS;
-  if (!make_map(&mK64, k, 64, N, BH, 64) || !make_map(&mV64, v, 64, N, BH, 64) ||
+  const int G = (int)std::max<size_t>(1, std::min<size_t>(BH, budget / per_head));
+  int st = SATA_OK;
+  uint8_t *ws = (uint8_t *)get_workspace(stream, per_head * G + 256, &st);
+  if (!ws) return st;
+  __nv_bfloat16 *kt = reinterpret_cast<__nv_bfloat16 *>(ws);
+  __nv_bfloat16 *snap =
+      reinterpret_cast<__nv_bfloat16 *>(ws + ((kt_head * G + 255) & ~(size_t)255));
+  CUtensorMap mV64, mQ, mK64, mS, mKT;
+  if (!make_map(&mV64, v, 64, N, BH, 64) || !make_map(&mK64, k, 64, N, BH, 64) ||
       !make_map(&mQ, q, 64, N, BH, 128))
     return SATA_ERR_CUDA;
   static bool attr_done = false;
@@ -643,19 +690,24 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
 
-  const int n_mt = n_tiles / 2;
+  const int n_mt = m_pad / 128;
   const int n_batches = (n_mt + kUF - 1) / kUF;
-  const GenWeights W = weights64();
+  GenWeights ones;  // the readout generates unweighted monomials
+  ones.w3 = ones.w3h = ones.w3s = ones.w2 = ones.w2h = ones.w1 = 1.f;
   for (int h0 = 0; h0 < BH; h0 += G) {
     const int g = std::min(G, BH - h0);
-    if (nsnap > 0 &&
-        !make_map(&mS, snap, (uint64_t)m_pad, 65, (uint64_t)g * nsnap, kNP))
+    if (!make_map(&mKT, kt, (uint64_t)Npad, 65, (uint64_t)g, 65)) return SATA_ERR_CUDA;
+    if (nsnap > 0 && !make_map(&mS, snap, (uint64_t)m_pad, 65, (uint64_t)g * nsnap, kNP))
       return SATA_ERR_CUDA;
+    prof_kernel_begin(stream, K_TC_PREP);
+    tc_transpose_k<<<dim3(Npad / 64, g), 256, 0, stream>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(k), kt, N, Npad, h0);
+    prof_kernel_end(stream);
     UParams up;
-    up.tiles = reinterpret_cast<const TileDesc *>(basis->tile_desc);
+    up.slot_idx = basis->slot_idx;
+    up.slot_w = basis->slot_w;
     up.row_of_slot = basis->tile_row;
-    up.W = W;
-    up.n_tiles = n_tiles;
+    up.n_mt = n_mt;
     up.N = N;
     up.C = C;
     up.nsnap = nsnap;
@@ -668,11 +720,11 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
     up.state = state;
     up.err = err;
     prof_kernel_begin(stream, K_TC_CHUNK_STATES);
-    tc_chunk_states<<<std::min(up.n_items, nsm), kThreads, kUSmem, stream>>>(mK64, mV64, up);
+    tc_chunk_states<<<std::min(up.n_items, nsm), kUThreads, kUSmem, stream>>>(mKT, mV64, up);
     prof_kernel_end(stream);
     RParams rp;
-    rp.tiles = up.tiles;
-    rp.W = W;
+    rp.tiles = reinterpret_cast<const TileDesc *>(basis->tile_desc);
+    rp.W = ones;
     rp.n_tiles = n_tiles;
     rp.N = N;
     rp.C = C;

@@ -46,6 +46,8 @@ void free_basis(DeviceBasis *b) {
   cudaFree(b->w);
   cudaFree(b->tile_desc);
   cudaFree(b->tile_row);
+  cudaFree(b->slot_idx);
+  cudaFree(b->slot_w);
   delete b;
 }
 
@@ -89,7 +91,28 @@ const DeviceBasis *get_device_basis(int dK, int P, int *status) {
     }
     db->n_tiles = to.n_tiles;
     db->m_pad = (int64_t)to.n_tiles * 64;
-    ok = cudaMalloc(&db->tile_desc, to.tiles.size() * sizeof(TileDesc)) == cudaSuccess &&
+    // per slot: the row's index triple (unused slots point at row 64, the ones
+    // row of the transposed keys) and its weight
+    std::vector<uint32_t> sidx(db->m_pad, 0x404040u);
+    std::vector<float> sw(db->m_pad, 0.f);
+    for (int64_t k = 0; k < db->m_pad; ++k) {
+      const int32_t r = to.row_of_slot[k];
+      if (r < 0) continue;
+      uint32_t v = 0;
+      for (int q = 0; q < 3; ++q) {
+        const int ii = q < hb.degree[r] ? hb.ix[3 * r + q] : 64;
+        v |= (uint32_t)ii << (8 * q);
+      }
+      sidx[k] = v;
+      sw[k] = (float)hb.weight[r];
+    }
+    ok = cudaMalloc(&db->slot_idx, sidx.size() * sizeof(uint32_t)) == cudaSuccess &&
+         cudaMalloc(&db->slot_w, sw.size() * sizeof(float)) == cudaSuccess &&
+         cudaMemcpy(db->slot_idx, sidx.data(), sidx.size() * sizeof(uint32_t),
+                    cudaMemcpyHostToDevice) == cudaSuccess &&
+         cudaMemcpy(db->slot_w, sw.data(), sw.size() * sizeof(float), cudaMemcpyHostToDevice) ==
+             cudaSuccess &&
+         cudaMalloc(&db->tile_desc, to.tiles.size() * sizeof(TileDesc)) == cudaSuccess &&
          cudaMalloc(&db->tile_row, to.row_of_slot.size() * sizeof(int32_t)) == cudaSuccess &&
          cudaMemcpy(db->tile_desc, to.tiles.data(), to.tiles.size() * sizeof(TileDesc),
                     cudaMemcpyHostToDevice) == cudaSuccess &&

@@ -38,6 +38,8 @@ struct DeviceBasis {
   int64_t m_pad = 0;            // n_tiles * 64
   void *tile_desc = nullptr;      // [n_tiles] TileDesc (tile_order.h)
   int32_t *tile_row = nullptr;    // [m_pad] lexicographic row of each padded feature (-1 = pad)
+  uint32_t *slot_idx = nullptr;   // [m_pad] i | j << 8 | l << 16 of each slot (unused = 64)
+  float *slot_w = nullptr;        // [m_pad] basis weight of each slot (0 = pad)
 };
 
 // Returns the cached tables for the current device (builds them on first use).

@@ -9,8 +9,8 @@
 // Arithmetic (feature = w_alpha * prod x): OUTER and BC tiles form the pair
 // product u = w * x_i * x_j in fp32, round it to bf16 and multiply by the
 // eight values of the third octet with packed bf16x2 multiplies (two
-// roundings); D and MISC tiles (21 of 749) form each product in fp32 and round
-// once.
+// roundings); D and MISC tiles (21 of 749) load the octets they touch once and
+// form each product in fp32, rounding once.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -149,41 +149,64 @@ SATA_HD void gen_bc(const TileDesc &td, const uint8_t *row, uint32_t rsw,
   bc_variant<T>(g0, r0, g1, r1, W, out, std::make_integer_sequence<int, 8>{});
 }
 
-// ---- D: features 64*T + P of the concatenated in-octet triples
+// ---- D: features 64*T + P of the concatenated in-octet triples; a tile
+// touches at most two octets, loaded once (ga = first, gb = second).
+template <int T> struct DOctets {
+  static constexpr int ga = (64 * T) / 120;
+  static constexpr int gb = (64 * T + 63) / 120 < 8 ? (64 * T + 63) / 120 : 7;
+};
+
 template <int T, int P>
-SATA_HD float d_feature(const uint8_t *row, uint32_t rsw, const GenWeights &W) {
+SATA_HD float d_feature(const float (&xa)[8], const float (&xb)[8], const GenWeights &W) {
   constexpr int f = 64 * T + P;
   if constexpr (f >= 120 * 8) {
     return 0.f;
   } else {
     constexpr int g = f / 120, r = f % 120;
-    constexpr int a = 8 * g + triple_at(r, 0), b = 8 * g + triple_at(r, 1),
-                  c = 8 * g + triple_at(r, 2);
+    constexpr int a = triple_at(r, 0), b = triple_at(r, 1), c = triple_at(r, 2);
     constexpr int fa = fact3(a, b, c);
     const float w = fa == 1 ? W.w3 : fa == 2 ? W.w3h : W.w3s;
-    return w * load_elem(row, rsw, a) * load_elem(row, rsw, b) * load_elem(row, rsw, c);
+    const float(&x)[8] = (g == DOctets<T>::ga) ? xa : xb;
+    return w * x[a] * x[b] * x[c];
   }
 }
 
 template <int T, int... Q>
 SATA_HD void d_variant(const uint8_t *row, uint32_t rsw, const GenWeights &W,
-                                          uint32_t (&out)[32], std::integer_sequence<int, Q...>) {
-  ((out[Q] = pack2(d_feature<T, 2 * Q>(row, rsw, W), d_feature<T, 2 * Q + 1>(row, rsw, W))),
-   ...);
+                       uint32_t (&out)[32], std::integer_sequence<int, Q...>) {
+  float xa[8], xb[8];
+  unpack8(load_chunk(row, rsw, DOctets<T>::ga), xa);
+  unpack8(load_chunk(row, rsw, DOctets<T>::gb), xb);
+  ((out[Q] = pack2(d_feature<T, 2 * Q>(xa, xb, W), d_feature<T, 2 * Q + 1>(xa, xb, W))), ...);
 }
 
-// ---- MISC: in-octet pairs (degree 2), degree 1, degree 0, padding
+// ---- MISC: in-octet pairs (degree 2), degree 1, degree 0, padding.  The
+// octets a tile needs are loaded once into registers (mask of octets).
+template <int T> struct MiscOctets {
+  static constexpr int n2 = 36 * 8, n1 = 64;
+  static constexpr int octet_of(int f) {
+    return f < n2 ? f / 36 : (f < n2 + n1 ? (f - n2) / 8 : -1);
+  }
+  static constexpr unsigned mask() {
+    unsigned m = 0;
+    for (int p = 0; p < 64; ++p) {
+      const int g = octet_of(64 * T + p);
+      if (g >= 0) m |= 1u << g;
+    }
+    return m;
+  }
+};
+
 template <int T, int P>
-SATA_HD float misc_feature(const uint8_t *row, uint32_t rsw,
-                                              const GenWeights &W) {
+SATA_HD float misc_feature(const float (&xo)[8][8], const GenWeights &W) {
   constexpr int f = 64 * T + P;
   constexpr int n2 = 36 * 8, n1 = 64;
   if constexpr (f < n2) {
     constexpr int g = f / 36, pr = f % 36;
-    constexpr int a = 8 * g + pair_a(pr), b = 8 * g + pair_b(pr);
-    return (a == b ? W.w2h : W.w2) * load_elem(row, rsw, a) * load_elem(row, rsw, b);
+    constexpr int a = pair_a(pr), b = pair_b(pr);
+    return (a == b ? W.w2h : W.w2) * xo[g][a] * xo[g][b];
   } else if constexpr (f < n2 + n1) {
-    return W.w1 * load_elem(row, rsw, f - n2);
+    return W.w1 * xo[(f - n2) / 8][(f - n2) % 8];
   } else if constexpr (f == n2 + n1) {
     return 1.f;
   } else {
@@ -191,13 +214,18 @@ SATA_HD float misc_feature(const uint8_t *row, uint32_t rsw,
   }
 }
 
+template <int T, int... G>
+SATA_HD void misc_load(const uint8_t *row, uint32_t rsw, float (&xo)[8][8],
+                       std::integer_sequence<int, G...>) {
+  (((MiscOctets<T>::mask() >> G) & 1u ? unpack8(load_chunk(row, rsw, G), xo[G]) : void()), ...);
+}
+
 template <int T, int... Q>
-SATA_HD void misc_variant(const uint8_t *row, uint32_t rsw,
-                                             const GenWeights &W, uint32_t (&out)[32],
-                                             std::integer_sequence<int, Q...>) {
-  ((out[Q] = pack2(misc_feature<T, 2 * Q>(row, rsw, W),
-                         misc_feature<T, 2 * Q + 1>(row, rsw, W))),
-   ...);
+SATA_HD void misc_variant(const uint8_t *row, uint32_t rsw, const GenWeights &W,
+                          uint32_t (&out)[32], std::integer_sequence<int, Q...>) {
+  float xo[8][8];
+  misc_load<T>(row, rsw, xo, std::make_integer_sequence<int, 8>{});
+  ((out[Q] = pack2(misc_feature<T, 2 * Q>(xo, W), misc_feature<T, 2 * Q + 1>(xo, W))), ...);
 }
 
 // Generates tile td for the token whose swizzled row starts at `row`
