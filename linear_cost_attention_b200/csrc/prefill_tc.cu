@@ -71,21 +71,22 @@ __device__ __forceinline__ void fill_ones(uint8_t *blk, int rows) {
 // accumulates S' += m(K)^T [V, 1]; the basis weights are applied when S' leaves
 // TMEM: state = w S', snapshot = w^2 S' (the readout then multiplies by the
 // unweighted m(q): sum_a w_a m_a(q) w_a S'_a = phi(q) . S).
-constexpr int kUF = 3;          // 128-row state tiles per item
-constexpr int kUT = 64;         // tokens per step
+constexpr int kUF = 2;          // 128-row state tiles per item
+constexpr int kUT = 128;        // tokens per step
 constexpr int kUAS = 2;         // A stages (TMEM)
-constexpr int kUKS = 6;         // K^T / V stages (shared memory)
+constexpr int kUKS = 4;         // K^T / V stages (shared memory)
 constexpr int kUGenWarps = 4 * kUF;
 constexpr int kUThreads = 32 * (2 + kUGenWarps);
 constexpr int kMaxTiles = 768;  // tile table capacity in smem (readout)
-constexpr uint32_t kUColA = 256;               // TMEM: D at f*80, A from column 256
+constexpr uint32_t kUColA = 160;               // TMEM: D at f*80, A from column 160
 constexpr uint32_t kUTmemCols = 512;
-constexpr uint32_t kUKT = 9 * 1024;            // 65 rows x 128 B, padded to 9 KiB
-constexpr uint32_t kUV = kUT * kRow;           // 8 KiB
+constexpr uint32_t kUKTh = 9 * 1024;           // one 64-token K^T box: 65 rows x 128 B, padded
+constexpr uint32_t kUKT = 2 * kUKTh;           // K^T of one step (two boxes)
+constexpr uint32_t kUV = kUT * kRow;           // 16 KiB
 constexpr uint32_t kUOffKT = 0, kUOffV = kUOffKT + kUKS * kUKT, kUOffOnes = kUOffV + kUKS * kUV,
                    kUOffBar = kUOffOnes + kUV;
 constexpr uint32_t kUSmem = kUOffBar + 256 + 1024;
-static_assert(kUColA + kUAS * kUF * 32 <= 512 && kUF * kNP <= kUColA, "TMEM budget");
+static_assert(kUColA + kUAS * kUF * (kUT / 2) <= kUTmemCols && kUF * kNP <= kUColA, "TMEM budget");
 
 struct UParams {
   const uint32_t *slot_idx;  // [m_pad] i | j << 8 | l << 16 (64 = the ones row)
@@ -155,8 +156,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
           if (it >= kUKS &&
               !(ok = mbar_wait(&kv_empty[st], ((it / kUKS) - 1) & 1, abort_flag, p.err)))
             break;
-          mbar_arrive_expect_tx(&kv_full[st], 65 * kRow + kUV);
+          mbar_arrive_expect_tx(&kv_full[st], 2 * 65 * kRow + kUV);
           tma_load_3d(sKT + st * kUKT, &tmKT, &kv_full[st], s * kUT, 0, hb);
+          tma_load_3d(sKT + st * kUKT + kUKTh, &tmKT, &kv_full[st], s * kUT + 64, 0, hb);
           tma_load_3d(sV + st * kUV, &tmV, &kv_full[st], 0, s * kUT, bh);
         }
       }
@@ -190,7 +192,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
               tc_fence_after();
             }
             if (f >= nmt) continue;
-            const uint32_t a0 = tmem + kUColA + (as * kUF + f) * 32;
+            const uint32_t a0 = tmem + kUColA + (as * kUF + f) * (kUT / 2);
 #pragma unroll
             for (int k = 0; k < kUT / 16; ++k) {
               const uint64_t bd = smem_desc_sw128(v0 + k * 2048, lbo_b, 1024);
@@ -280,19 +282,22 @@ __global__ void __launch_bounds__(kUThreads, 1)
         if (it >= kUAS &&
             !(ok = mbar_wait(&a_empty[as], ((it / kUAS) - 1) & 1, abort_flag, p.err)))
           break;
-        const uint8_t *kt = sKT + ks * kUKT;
-        uint32_t out[32];
+#pragma unroll 1
+        for (int h = 0; h < kUT / 64; ++h) {  // 64 tokens (one K^T box) at a time
+          const uint8_t *kt = sKT + ks * kUKT + h * kUKTh;
+          uint32_t out[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 xi = *reinterpret_cast<const uint4 *>(kt + ri + (((uint32_t)c ^ si) << 4));
-          const uint4 xj = *reinterpret_cast<const uint4 *>(kt + rj + (((uint32_t)c ^ sj) << 4));
-          const uint4 xl = *reinterpret_cast<const uint4 *>(kt + rl + (((uint32_t)c ^ sl) << 4));
-          out[4 * c + 0] = bmul2(bmul2(xi.x, xj.x), xl.x);
-          out[4 * c + 1] = bmul2(bmul2(xi.y, xj.y), xl.y);
-          out[4 * c + 2] = bmul2(bmul2(xi.z, xj.z), xl.z);
-          out[4 * c + 3] = bmul2(bmul2(xi.w, xj.w), xl.w);
+          for (int c = 0; c < 8; ++c) {
+            const uint4 xi = *reinterpret_cast<const uint4 *>(kt + ri + (((uint32_t)c ^ si) << 4));
+            const uint4 xj = *reinterpret_cast<const uint4 *>(kt + rj + (((uint32_t)c ^ sj) << 4));
+            const uint4 xl = *reinterpret_cast<const uint4 *>(kt + rl + (((uint32_t)c ^ sl) << 4));
+            out[4 * c + 0] = bmul2(bmul2(xi.x, xj.x), xl.x);
+            out[4 * c + 1] = bmul2(bmul2(xi.y, xj.y), xl.y);
+            out[4 * c + 2] = bmul2(bmul2(xi.z, xj.z), xl.z);
+            out[4 * c + 3] = bmul2(bmul2(xi.w, xj.w), xl.w);
+          }
+          tmem_st32(tmem + tl + kUColA + (as * kUF + f) * (kUT / 2) + 32 * h, out);
         }
-        tmem_st32(tmem + tl + kUColA + (as * kUF + f) * 32, out);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -335,17 +340,18 @@ __global__ void __launch_bounds__(256) tc_transpose_k(const __nv_bfloat16 *__res
 }
 
 // ============================================================ readout
-constexpr int kRStages = 10;             // phi(Q) stages, in TMEM (32 columns each)
-constexpr int kRBS = 12;                 // snapshot-tile stages (cover TMA latency)
+constexpr int kRTS = 3;                  // feature tiles per pipeline stage
+constexpr int kRStages = 3;              // phi(Q) stages, in TMEM (32 columns per tile)
+constexpr int kRBS = 4;                  // snapshot stages (kRTS tiles each)
 constexpr int kKB = 64;                  // keys per in-chunk block
 constexpr uint32_t kRTile = 128 * kRow;  // 128 tokens x 64 features: 16 KiB
 constexpr uint32_t kRB = kNP * kRow;     // 80 x 64 snapshot tile: 10 KiB
 constexpr uint32_t kRKV = kKB * kRow;    // 64 keys x 64: 8 KiB
 constexpr uint32_t kRColS = 96, kRColA = 160;  // TMEM: D 0..79, scores 96..159, A stages
 constexpr uint32_t kRTmemCols = 512;
-static_assert(kRColA + 32 * kRStages <= kRTmemCols, "TMEM budget");
+static_assert(kRColA + 32 * kRTS * kRStages <= kRTmemCols, "TMEM budget");
 constexpr uint32_t kROffQ = 0, kROffB = kROffQ + kRTile,
-                   kROffK = kROffB + kRBS * kRB, kROffV = kROffK + kRKV,
+                   kROffK = kROffB + kRBS * kRTS * kRB, kROffV = kROffK + kRKV,
                    kROffOnes = kROffV + kRKV, kROffP = kROffOnes + kRKV,
                    kROffTiles = kROffP + 2 * kRTile, kROffBar = kROffTiles + kMaxTiles * 8;
 constexpr uint32_t kRSmem = kROffBar + 512 + 1024;  // 50 barriers + TMEM slot + flag
@@ -422,13 +428,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- TMA producer: snapshot tiles S_(c-1)[80 x 64 rows]
     if (lane == 0 && inter) {
       prefetch_tensormap(&tmS);
+      const int n_stages = (p.n_tiles + kRTS - 1) / kRTS;
       int i = 0;
-      for (; i < p.n_tiles; ++i) {
+      for (; i < n_stages; ++i) {
         const int st = i % kRBS;
         if (i >= kRBS && !mbar_wait(&b_empty[st], ((i / kRBS) - 1) & 1, abort_flag, p.err))
           break;
-        mbar_arrive_expect_tx(&b_full[st], kRB);
-        tma_load_3d(sB + st * kRB, &tmS, &b_full[st], 64 * i, 0, hrel * p.nsnap + chunk - 1);
+        const int nt = min(kRTS, p.n_tiles - kRTS * i);
+        mbar_arrive_expect_tx(&b_full[st], nt * kRB);
+        for (int t = 0; t < nt; ++t)
+          tma_load_3d(sB + (st * kRTS + t) * kRB, &tmS, &b_full[st], 64 * (kRTS * i + t), 0,
+                      hrel * p.nsnap + chunk - 1);
       }
       for (int j = max(0, i - kRBS); j < i; ++j) {
         volatile int never = 0;
@@ -504,17 +514,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) intra(false);
       if (ok && inter) {
         const uint32_t b0 = smem_u32(sB);
-        for (int i = 0; i < p.n_tiles; ++i) {
+        const int n_stages = (p.n_tiles + kRTS - 1) / kRTS;
+        for (int i = 0; i < n_stages; ++i) {
           const int st = i % kRStages, bs = i % kRBS;
           if (!(ok = mbar_wait(&a_full[st], (i / kRStages) & 1, abort_flag, p.err))) break;
           if (!(ok = mbar_wait(&b_full[bs], (i / kRBS) & 1, abort_flag, p.err))) break;
           tc_fence_after();
+          const int nt = min(kRTS, p.n_tiles - kRTS * i);
+          for (int t = 0; t < nt; ++t) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16_ts(tD, tmem + kRColA + st * 32 + 8 * k,
-                        smem_desc_sw128(b0 + bs * kRB + 32 * k, 16, 1024), id_inter,
-                        (d_init || k > 0) ? 1u : 0u);
-          d_init = true;
+            for (int k = 0; k < 4; ++k)
+              mma_bf16_ts(tD, tmem + kRColA + (st * kRTS + t) * 32 + 8 * k,
+                          smem_desc_sw128(b0 + (bs * kRTS + t) * kRB + 32 * k, 16, 1024),
+                          id_inter, (d_init || k > 0) ? 1u : 0u);
+            d_init = true;
+          }
           mma_commit(&a_empty[st]);
           mma_commit(&b_empty[bs]);
           intra(false);
@@ -588,17 +602,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = lane + 32 * (gw & 3);
     bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
     const uint8_t *qrow = sQ + row * kRow;
-    for (int i = half; ok && i < p.n_tiles; i += 2) {
+    const int n_stages = (p.n_tiles + kRTS - 1) / kRTS;
+    for (int i = half; ok && i < n_stages; i += 2) {
       const int st = i % kRStages;
       if (i >= kRStages && !(ok = mbar_wait(&a_empty[st], ((i / kRStages) - 1) & 1, abort_flag,
                                             p.err)))
         break;
-      const TileDesc td = sTiles[i];
-      uint32_t out[32];
-      gen_tile(td, qrow, (uint32_t)(row & 7), p.W, out);
-      // this thread's token is TMEM lane `row`; the tile's 64 features are 32
-      // packed columns of stage st
-      tmem_st32(tmem + ((uint32_t)(32 * (gw & 3)) << 16) + kRColA + st * 32, out);
+#pragma unroll 1
+      for (int t = 0; t < kRTS; ++t) {
+        const int ti = kRTS * i + t;
+        uint32_t out[32];
+        if (ti < p.n_tiles) {
+          const TileDesc td = sTiles[ti];
+          gen_tile(td, qrow, (uint32_t)(row & 7), p.W, out);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) out[q] = 0u;
+        }
+        // this thread's token is TMEM lane `row`; a tile's 64 features are 32
+        // packed columns
+        tmem_st32(tmem + ((uint32_t)(32 * (gw & 3)) << 16) + kRColA + (st * kRTS + t) * 32, out);
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -661,7 +685,7 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
   const int m_pad = n_tiles * 64;
   const int C = N <= 1024 ? ((N + 127) / 128) * 128 : 1024;
   const int nsnap = (N + C - 1) / C - 1;
-  const int Npad = ((N + kUT - 1) / kUT) * kUT;
+  const int Npad = ((N + kUT - 1) / kUT) * kUT;  // multiple of the 128-token step
   const size_t snap_head = (size_t)nsnap * 65 * m_pad * 2;
   const size_t kt_head = (size_t)65 * Npad * 2;
   const size_t per_head = snap_head + kt_head;
@@ -673,9 +697,9 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
   __nv_bfloat16 *kt = reinterpret_cast<__nv_bfloat16 *>(ws);
   __nv_bfloat16 *snap =
       reinterpret_cast<__nv_bfloat16 *>(ws + ((kt_head * G + 255) & ~(size_t)255));
-  CUtensorMap mV64, mQ, mK64, mS, mKT;
+  CUtensorMap mV64, mVU, mQ, mK64, mS, mKT;
   if (!make_map(&mV64, v, 64, N, BH, 64) || !make_map(&mK64, k, 64, N, BH, 64) ||
-      !make_map(&mQ, q, 64, N, BH, 128))
+      !make_map(&mVU, v, 64, N, BH, kUT) || !make_map(&mQ, q, 64, N, BH, 128))
     return SATA_ERR_CUDA;
   static bool attr_done = false;
   if (!attr_done) {
@@ -720,7 +744,7 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
     up.state = state;
     up.err = err;
     prof_kernel_begin(stream, K_TC_CHUNK_STATES);
-    tc_chunk_states<<<std::min(up.n_items, nsm), kUThreads, kUSmem, stream>>>(mKT, mV64, up);
+    tc_chunk_states<<<std::min(up.n_items, nsm), kUThreads, kUSmem, stream>>>(mKT, mVU, up);
     prof_kernel_end(stream);
     RParams rp;
     rp.tiles = reinterpret_cast<const TileDesc *>(basis->tile_desc);
