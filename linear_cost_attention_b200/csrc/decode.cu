@@ -33,7 +33,7 @@ template <> struct DecodeShape<17> { static constexpr int KB = 15; };  // 255
 template <> struct DecodeShape<9> { static constexpr int KB = 28; };   // 252
 
 template <int D1, typename T>
-__global__ void __launch_bounds__(D1 *DecodeShape<D1>::KB, 3)
+__global__ void __launch_bounds__(D1 *DecodeShape<D1>::KB)
     decode_stream(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                   float *__restrict__ state, const uint32_t *__restrict__ idx,
                   const float *__restrict__ w, int m, int dK, long long E, float *__restrict__ y) {
@@ -42,9 +42,11 @@ __global__ void __launch_bounds__(D1 *DecodeShape<D1>::KB, 3)
   constexpr int PER_IT = 4 * NT;
   constexpr int ROWS_IT = 4 * KB;
   constexpr long long L = (long long)PER_IT * kIters;
-  constexpr int MAXROWS = ROWS_IT * kIters + 2;
+  constexpr int MAXROWS = ROWS_IT * kIters + 1;
   constexpr int DV = D1 - 1;
-  __shared__ float2 s_f[MAXROWS];  // (phi_r(q), phi_r(k)) of the rows this block touches
+  __shared__ float s_fq[MAXROWS];
+  __shared__ float s_fk[MAXROWS];
+  __shared__ int s_bh[MAXROWS];
   __shared__ float s_y[2][D1];
 
   const int tid = threadIdx.x;
@@ -53,9 +55,6 @@ __global__ void __launch_bounds__(D1 *DecodeShape<D1>::KB, 3)
   const long long r_first = e_begin / D1;  // e_begin is a multiple of D1
   const int nrows = (int)((e_end - 1) / D1 - r_first + 1);
   const int head_first = (int)(r_first / m);
-  const int head_last = (int)(((e_end - 1) / D1) / m);
-  // first block-relative row of the second head (beyond the block if none)
-  const int split_row = (int)min((long long)MAXROWS, (long long)(head_first + 1) * m - r_first);
 
   for (int i = tid; i < nrows; i += NT) {
     const long long r = r_first + i;
@@ -69,105 +68,84 @@ __global__ void __launch_bounds__(D1 *DecodeShape<D1>::KB, 3)
       fq *= to_f32(q[(size_t)bh * dK + ii]);
       fk *= to_f32(k[(size_t)bh * dK + ii]);
     }
-    s_f[i] = make_float2(fq, fk);
+    s_fq[i] = fq;
+    s_fk[i] = fk;
+    s_bh[i] = bh;
   }
-  if (tid < 2) s_f[nrows + tid] = make_float2(0.f, 0.f);
   for (int i = tid; i < 2 * D1; i += NT) (&s_y[0][0])[i] = 0.f;
   __syncthreads();
 
-  // this thread's 4 elements of every iteration: fixed columns, rows rof0 or
-  // rof0 + 1 (element u sits in the second row when u >= usplit)
-  int col[4];
-  const int rof0 = (4 * tid) / D1;
-  int usplit = 4;
+  int col[4], rof[4], cur[4];
+  float acc[4], vv[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     col[u] = (4 * tid + u) % D1;
-    if (usplit == 4 && (4 * tid + u) / D1 != rof0) usplit = u;
+    rof[u] = (4 * tid + u) / D1;
+    cur[u] = -1;
+    acc[u] = 0.f;
+    vv[u] = 0.f;
   }
-  float acc0[4], acc1[4], vv0[4], vv1[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    acc0[u] = 0.f;
-    acc1[u] = 0.f;
-    vv0[u] = (col[u] < DV) ? to_f32(v[(size_t)head_first * DV + col[u]]) : 1.f;
-    vv1[u] = (col[u] < DV && head_first + 1 <= head_last)
-                 ? to_f32(v[(size_t)(head_first + 1) * DV + col[u]])
-                 : 1.f;
-  }
-  // rows of a third or later head (blocks that span more than two heads, only
-  // when m is small) take the general path below
-  const bool simple = head_last <= head_first + 1;
 
+  auto flush = [&](int u) {
+    if (cur[u] < 0) return;
+    if (cur[u] == head_first)
+      atomicAdd(&s_y[0][col[u]], acc[u]);
+    else if (cur[u] == head_first + 1)
+      atomicAdd(&s_y[1][col[u]], acc[u]);
+    else
+      atomicAdd(&y[(size_t)cur[u] * D1 + col[u]], acc[u]);
+    acc[u] = 0.f;
+  };
+
+  // kUnroll iterations at a time: all their 16-byte loads are issued before any
+  // is used, so each thread keeps kUnroll*16 bytes in flight.
   for (int it0 = 0; it0 < kIters; it0 += kUnroll) {
-    float sv[kUnroll][4];
+    float s[kUnroll][4];
     long long e[kUnroll];
 #pragma unroll
     for (int j = 0; j < kUnroll; ++j) {
       e[j] = e_begin + (long long)(it0 + j) * PER_IT + 4 * tid;
       if (e[j] + 3 < e_end) {
         const float4 x = __ldcs(reinterpret_cast<const float4 *>(state + e[j]));
-        sv[j][0] = x.x; sv[j][1] = x.y; sv[j][2] = x.z; sv[j][3] = x.w;
+        s[j][0] = x.x; s[j][1] = x.y; s[j][2] = x.z; s[j][3] = x.w;
       } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) sv[j][u] = (e[j] + u < e_end) ? state[e[j] + u] : 0.f;
+        for (int u = 0; u < 4; ++u) s[j][u] = (e[j] + u < e_end) ? state[e[j] + u] : 0.f;
       }
     }
 #pragma unroll
     for (int j = 0; j < kUnroll; ++j) {
       if (e[j] >= e_end) break;
       const bool full = (e[j] + 3 < e_end);
-      const int r0 = (it0 + j) * ROWS_IT + rof0;
-      const float2 f0 = s_f[r0], f1 = s_f[r0 + 1];
-      if (simple) {
+      const int rbase = (it0 + j) * ROWS_IT;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (!full && e[j] + u >= e_end) continue;  // past the end of the array
-          const int rr = u < usplit ? r0 : r0 + 1;
-          const float2 f = u < usplit ? f0 : f1;
-          const bool second = rr >= split_row;
-          const float sn = fmaf(f.y, second ? vv1[u] : vv0[u], sv[j][u]);
-          sv[j][u] = sn;
-          if (second)
-            acc1[u] = fmaf(f.x, sn, acc1[u]);
-          else
-            acc0[u] = fmaf(f.x, sn, acc0[u]);
+      for (int u = 0; u < 4; ++u) {
+        if (!full && e[j] + u >= e_end) continue;  // past the end of the array
+        const int rr = min(rbase + rof[u], nrows - 1);
+        const int bh = s_bh[rr];
+        if (bh != cur[u]) {
+          flush(u);
+          cur[u] = bh;
+          vv[u] = (col[u] < DV) ? to_f32(v[(size_t)bh * DV + col[u]]) : 1.f;
         }
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (!full && e[j] + u >= e_end) continue;
-          const int rr = u < usplit ? r0 : r0 + 1;
-          const float2 f = u < usplit ? f0 : f1;
-          const int bh = (int)((r_first + rr) / m);
-          const float vu = (col[u] < DV) ? to_f32(v[(size_t)bh * DV + col[u]]) : 1.f;
-          const float sn = fmaf(f.y, vu, sv[j][u]);
-          sv[j][u] = sn;
-          const float contrib = f.x * sn;
-          if (bh == head_first)
-            acc0[u] += contrib;
-          else if (bh == head_first + 1)
-            acc1[u] += contrib;
-          else
-            atomicAdd(&y[(size_t)bh * D1 + col[u]], contrib);
-        }
+        const float sn = fmaf(s_fk[rr], vv[u], s[j][u]);
+        s[j][u] = sn;
+        acc[u] = fmaf(s_fq[rr], sn, acc[u]);
       }
       if (full) {
         __stcs(reinterpret_cast<float4 *>(state + e[j]),
-               make_float4(sv[j][0], sv[j][1], sv[j][2], sv[j][3]));
+               make_float4(s[j][0], s[j][1], s[j][2], s[j][3]));
       } else {
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          if (e[j] + u < e_end) state[e[j] + u] = sv[j][u];
+          if (e[j] + u < e_end) state[e[j] + u] = s[j][u];
       }
     }
   }
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    atomicAdd(&s_y[0][col[u]], acc0[u]);
-    atomicAdd(&s_y[1][col[u]], acc1[u]);
-  }
+  for (int u = 0; u < 4; ++u) flush(u);
   __syncthreads();
+  const int head_last = s_bh[nrows - 1];
   for (int i = tid; i < 2 * D1; i += NT) {
     const int slot = i / D1, c = i % D1;
     if (head_first + slot <= head_last)
