@@ -64,27 +64,29 @@ __device__ __forceinline__ void fill_ones(uint8_t *blk, int rows) {
 
 // ============================================================ chunk states
 // One CTA per (head, kUF x 128 basis rows).  Thread = basis row = TMEM lane:
-// each generator thread forms its row's unweighted monomial x_i x_j x_l for 64
-// tokens from the transposed keys (rows of K^T; index 64 is a row of ones that
-// is zero past the sequence end) and stores them with tcgen05.st straight into
-// the A operand in TMEM (basis rows x tokens, two tokens per column).  The MMA
-// accumulates S' += m(K)^T [V, 1]; the basis weights are applied when S' leaves
-// TMEM: state = w S', snapshot = w^2 S' (the readout then multiplies by the
-// unweighted m(q): sum_a w_a m_a(q) w_a S'_a = phi(q) . S).
+// each generator thread forms its row's unweighted monomial x_i x_j x_l for
+// the step's tokens from the transposed keys (rows of K^T; index 64 is a row of
+// ones that is zero past the sequence end) and stores them with tcgen05.st
+// straight into the A operand in TMEM (basis rows x tokens, two tokens per
+// column).  The MMA accumulates S' += m(K)^T [V, 1] with [V, 1]^T as a K-major
+// B operand (rows of V^T plus its ones row; rows 65..79 are TMA zero fill).  The
+// basis weights are applied when S' leaves TMEM: state = w S', snapshot =
+// w^2 S' (the readout then multiplies by the unweighted m(q):
+// sum_a w_a m_a(q) w_a S'_a = phi(q) . S).
 constexpr int kUF = 2;          // 128-row state tiles per item
 constexpr int kUT = 128;        // tokens per step
 constexpr int kUAS = 2;         // A stages (TMEM)
-constexpr int kUKS = 4;         // K^T / V stages (shared memory)
+constexpr int kUKS = 4;         // K^T / V^T stages (shared memory)
 constexpr int kUGenWarps = 4 * kUF;
-constexpr int kUThreads = 32 * (2 + kUGenWarps);
+constexpr int kUEpiWarp0 = 2, kUGenWarp0 = 6;  // warps 2..5 epilogue, 6.. generators
+constexpr int kUThreads = 32 * (kUGenWarp0 + kUGenWarps);
 constexpr int kMaxTiles = 768;  // tile table capacity in smem (readout)
 constexpr uint32_t kUColA = 160;               // TMEM: D at f*80, A from column 160
 constexpr uint32_t kUTmemCols = 512;
 constexpr uint32_t kUKTh = 9 * 1024;           // one 64-token K^T box: 65 rows x 128 B, padded
-constexpr uint32_t kUKT = 2 * kUKTh;           // K^T of one step (two boxes)
-constexpr uint32_t kUV = kUT * kRow;           // 16 KiB
-constexpr uint32_t kUOffKT = 0, kUOffV = kUOffKT + kUKS * kUKT, kUOffOnes = kUOffV + kUKS * kUV,
-                   kUOffBar = kUOffOnes + kUV;
+constexpr uint32_t kUVTh = kNP * kRow;         // one 64-token [V,1]^T box: 80 rows x 128 B
+constexpr uint32_t kUKT = 2 * kUKTh, kUVT = 2 * kUVTh;  // per step (two boxes each)
+constexpr uint32_t kUOffKT = 0, kUOffVT = kUOffKT + kUKS * kUKT, kUOffBar = kUOffVT + kUKS * kUVT;
 constexpr uint32_t kUSmem = kUOffBar + 256 + 1024;
 static_assert(kUColA + kUAS * kUF * (kUT / 2) <= kUTmemCols && kUF * kNP <= kUColA, "TMEM budget");
 
@@ -100,11 +102,11 @@ struct UParams {
 };
 
 __global__ void __launch_bounds__(kUThreads, 1)
-    tc_chunk_states(const __grid_constant__ CUtensorMap tmKT, const __grid_constant__ CUtensorMap tmV,
+    tc_chunk_states(const __grid_constant__ CUtensorMap tmKT, const __grid_constant__ CUtensorMap tmVT,
                     const UParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sKT = smem + kUOffKT, *sV = smem + kUOffV, *sOnes = smem + kUOffOnes;
+  uint8_t *sKT = smem + kUOffKT, *sVT = smem + kUOffVT;
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kUOffBar);
   uint64_t *kv_full = bar, *kv_empty = bar + kUKS, *a_full = bar + 2 * kUKS,
            *a_empty = a_full + kUAS, *snap_full = a_empty + kUAS, *snap_done = snap_full + 1,
@@ -128,8 +130,6 @@ __global__ void __launch_bounds__(kUThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  fill_ones(sOnes, kUT);
-  fence_proxy_async_smem();
   if (warp == 1) tmem_alloc(tmem_slot, kUTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -143,23 +143,24 @@ __global__ void __launch_bounds__(kUThreads, 1)
   };
 
   if (warp == 0) {
-    // ---------------- TMA producer: K^T (65 rows x 64 tokens) and V (64 x 64)
+    // ---------------- TMA producer: K^T (65 rows) and [V,1]^T (80 rows), 2 x 64 tokens
     if (lane == 0) {
       prefetch_tensormap(&tmKT);
-      prefetch_tensormap(&tmV);
+      prefetch_tensormap(&tmVT);
       uint32_t it = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int hb = item / p.n_batches, bh = p.head0 + hb;
+        const int hb = item / p.n_batches;
         for (int s = 0; s < nsub; ++s, ++it) {
           const int st = it % kUKS;
           if (it >= kUKS &&
               !(ok = mbar_wait(&kv_empty[st], ((it / kUKS) - 1) & 1, abort_flag, p.err)))
             break;
-          mbar_arrive_expect_tx(&kv_full[st], 2 * 65 * kRow + kUV);
-          tma_load_3d(sKT + st * kUKT, &tmKT, &kv_full[st], s * kUT, 0, hb);
-          tma_load_3d(sKT + st * kUKT + kUKTh, &tmKT, &kv_full[st], s * kUT + 64, 0, hb);
-          tma_load_3d(sV + st * kUV, &tmV, &kv_full[st], 0, s * kUT, bh);
+          mbar_arrive_expect_tx(&kv_full[st], 2 * 65 * kRow + 2 * kUVTh);
+          for (int h = 0; h < 2; ++h) {
+            tma_load_3d(sKT + st * kUKT + h * kUKTh, &tmKT, &kv_full[st], s * kUT + 64 * h, 0, hb);
+            tma_load_3d(sVT + st * kUVT + h * kUVTh, &tmVT, &kv_full[st], s * kUT + 64 * h, 0, hb);
+          }
         }
       }
       for (uint32_t j = it > kUKS ? it - kUKS : 0; j < it; ++j) {
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, kNP, false, true);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kNP, false, false);
       uint32_t it = 0, events = 0;
       bool after_event = false;
       bool ok = true;
@@ -182,8 +183,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
           if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err))) break;
           if (!(ok = mbar_wait(&a_full[as], (it / kUAS) & 1, abort_flag, p.err))) break;
           tc_fence_after();
-          const uint32_t v0 = smem_u32(sV + ks * kUV);
-          const uint32_t lbo_b = smem_u32(sOnes) - v0;
+          const uint32_t b0 = smem_u32(sVT + ks * kUVT);
           for (int f = 0; f < kUF; ++f) {
             // every tile's barrier is waited once per event, in order, so no
             // barrier can run two phases ahead of its waiter
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
             const uint32_t a0 = tmem + kUColA + (as * kUF + f) * (kUT / 2);
 #pragma unroll
             for (int k = 0; k < kUT / 16; ++k) {
-              const uint64_t bd = smem_desc_sw128(v0 + k * 2048, lbo_b, 1024);
+              const uint64_t bd = smem_desc_sw128(b0 + (k >> 2) * kUVTh + 32 * (k & 3), 16, 1024);
               mma_bf16_ts(tmem + f * kNP, a0 + 8 * k, bd, idesc, (s > 0 || k > 0) ? 1u : 0u);
             }
           }
@@ -214,68 +214,70 @@ __global__ void __launch_bounds__(kUThreads, 1)
       volatile int never = 0;
       mbar_wait(drain, 0, &never, p.err);
     }
+  } else if (warp >= kUEpiWarp0 && warp < kUGenWarp0) {
+    // ---------------- epilogue: S' -> snapshot (w^2 S') or state (w S')
+    const int q4 = warp & 3;
+    const int row = 32 * q4 + lane;
+    const uint32_t tl = (uint32_t)(32 * q4) << 16;
+    uint32_t events = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int hb = item / p.n_batches, batch = item % p.n_batches;
+      for (int s = 0; ok && s < nsub; ++s) {
+        if (!is_event(s)) continue;
+        if (!(ok = mbar_wait(snap_full, events & 1, abort_flag, p.err))) break;
+        ++events;
+        tc_fence_after();
+        const bool boundary = s != nsub - 1;
+        const int c = boundary ? (s + 1) / sub_per_chunk - 1 : 0;
+        for (int f = 0; f < kUF; ++f) {
+          const int mt = batch * kUF + f;
+          const bool live = mt < p.n_mt;
+          const int slot = mt * 128 + row;
+          const float w = live ? p.slot_w[slot] : 0.f;
+          const int r = (live && !boundary) ? p.row_of_slot[slot] : -1;
+          __nv_bfloat16 *sdst = p.snap + ((size_t)(hb * p.nsnap + c) * 65) * p.m_pad + slot;
+          float *tdst = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * 65;
+          const float scale = boundary ? w * w : w;
+          uint32_t v[kNP];
+          if (live) {
+#pragma unroll
+            for (int j = 0; j < kNP / 16; ++j)
+              tmem_ld16(tmem + tl + f * kNP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+            tmem_ld_wait();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&snap_done[f]);
+          if (!live) continue;
+          if (boundary) {
+#pragma unroll
+            for (int n = 0; n < 65; ++n)
+              sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(scale * __uint_as_float(v[n]));
+          } else if (r >= 0) {
+#pragma unroll
+            for (int n = 0; n < 65; ++n) tdst[n] = scale * __uint_as_float(v[n]);
+          }
+        }
+      }
+    }
   } else {
-    // ---------------- generators (one thread per basis row) and epilogue
-    const int g = warp - 2;
+    // ---------------- generators: one thread per basis row
+    const int g = warp - kUGenWarp0;
     const int f = g >> 2;               // state tile of this warp
     const int q4 = warp & 3;            // TMEM lane quarter
     const int row = 32 * q4 + lane;     // basis row inside the tile
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
-    uint32_t it = 0, events = 0;
+    uint32_t it = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int hb = item / p.n_batches, batch = item % p.n_batches;
+      const int batch = item % p.n_batches;
       const int mt = batch * kUF + f;
-      const bool live = mt < p.n_mt;
-      const int slot = mt * 128 + row;
       uint32_t ix = 0x404040u;  // three "ones" rows
-      float w = 0.f;
-      if (live) {
-        ix = p.slot_idx[slot];
-        w = p.slot_w[slot];
-      }
+      if (mt < p.n_mt) ix = p.slot_idx[mt * 128 + row];
       const uint32_t ri = (ix & 0xff) * kRow, rj = ((ix >> 8) & 0xff) * kRow,
                      rl = ((ix >> 16) & 0xff) * kRow;
       const uint32_t si = (ix & 7), sj = ((ix >> 8) & 7), sl = ((ix >> 16) & 7);
-      auto epilogue = [&](int s) {
-        // S' of this tile for this lane quarter -> snapshot (w^2 S') or state (w S')
-        if (!(ok = mbar_wait(snap_full, events & 1, abort_flag, p.err))) return;
-        ++events;
-        tc_fence_after();
-        // 16 columns at a time (65 used of the 80): load, scale, store
-        const bool boundary = s != nsub - 1;
-        const int c = boundary ? (s + 1) / sub_per_chunk - 1 : 0;
-        const int r = (live && !boundary) ? p.row_of_slot[slot] : -1;
-        __nv_bfloat16 *sdst = p.snap + ((size_t)(hb * p.nsnap + c) * 65) * p.m_pad + slot;
-        float *tdst = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * 65;
-        const float scale = boundary ? w * w : w;
-#pragma unroll 1
-        for (int j = 0; j < 5; ++j) {
-          uint32_t v[16];
-          if (live) {
-            tmem_ld16(tmem + tl + f * kNP + 16 * j, v);
-            tmem_ld_wait();
-          }
-          if (j == 4) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&snap_done[f]);
-          }
-          if (!live) continue;
-          const int nmax = j == 4 ? 1 : 16;  // column 64 is the last one used
-          if (boundary) {
-#pragma unroll
-            for (int n = 0; n < 16; ++n)
-              if (n < nmax)
-                sdst[(size_t)(16 * j + n) * p.m_pad] =
-                    __float2bfloat16_rn(scale * __uint_as_float(v[n]));
-          } else if (r >= 0) {
-#pragma unroll
-            for (int n = 0; n < 16; ++n)
-              if (n < nmax) tdst[16 * j + n] = scale * __uint_as_float(v[n]);
-          }
-        }
-      };
       for (int s = 0; ok && s < nsub; ++s, ++it) {
         const int ks = it % kUKS, as = it % kUAS;
         if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err))) break;
@@ -305,10 +307,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
           mbar_arrive(&a_full[as]);
           mbar_arrive(&kv_empty[ks]);
         }
-        // the previous step's snapshot, after this step's operand is handed over
-        if (s > 0 && is_event(s - 1)) epilogue(s - 1);
       }
-      if (ok && is_event(nsub - 1)) epilogue(nsub - 1);
     }
   }
 
@@ -318,24 +317,30 @@ __global__ void __launch_bounds__(kUThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kUTmemCols);
 }
 
-// K [BH, N, 64] -> K^T [BH, 65, Npad]: rows 0..63 the transposed keys, row 64
-// ones for t < N, zeros on the padding.
-__global__ void __launch_bounds__(256) tc_transpose_k(const __nv_bfloat16 *__restrict__ k,
-                                                      __nv_bfloat16 *__restrict__ kt, int N,
-                                                      int Npad, int head0) {
+// K [BH, N, 64] -> K^T [BH, 65, Npad] and V [BH, N, 64] -> V^T [BH, 65, Npad]:
+// rows 0..63 transposed, row 64 ones for t < N, zeros on the padding.
+__global__ void __launch_bounds__(256) tc_transpose_kv(const __nv_bfloat16 *__restrict__ k,
+                                                       const __nv_bfloat16 *__restrict__ v,
+                                                       __nv_bfloat16 *__restrict__ kt,
+                                                       __nv_bfloat16 *__restrict__ vt, int N,
+                                                       int Npad, int head0) {
   __shared__ __nv_bfloat16 tile[64][66];
   const int t0 = blockIdx.x * 64;
   const size_t bh = (size_t)head0 + blockIdx.y;
-  for (int e = threadIdx.x; e < 64 * 64; e += 256) {
-    const int t = e >> 6, d = e & 63;
-    tile[t][d] = (t0 + t < N) ? k[(bh * N + t0 + t) * 64 + d] : __float2bfloat16_rn(0.f);
-  }
-  __syncthreads();
-  __nv_bfloat16 *dst = kt + (size_t)blockIdx.y * 65 * Npad;
-  for (int e = threadIdx.x; e < 65 * 64; e += 256) {
-    const int d = e >> 6, t = e & 63;
-    dst[(size_t)d * Npad + t0 + t] =
-        d < 64 ? tile[t][d] : __float2bfloat16_rn(t0 + t < N ? 1.f : 0.f);
+  for (int which = 0; which < 2; ++which) {
+    const __nv_bfloat16 *src = which ? v : k;
+    __nv_bfloat16 *dst = (which ? vt : kt) + (size_t)blockIdx.y * 65 * Npad;
+    __syncthreads();
+    for (int e = threadIdx.x; e < 64 * 64; e += 256) {
+      const int t = e >> 6, d = e & 63;
+      tile[t][d] = (t0 + t < N) ? src[(bh * N + t0 + t) * 64 + d] : __float2bfloat16_rn(0.f);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < 65 * 64; e += 256) {
+      const int d = e >> 6, t = e & 63;
+      dst[(size_t)d * Npad + t0 + t] =
+          d < 64 ? tile[t][d] : __float2bfloat16_rn(t0 + t < N ? 1.f : 0.f);
+    }
   }
 }
 
@@ -687,19 +692,20 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
   const int nsnap = (N + C - 1) / C - 1;
   const int Npad = ((N + kUT - 1) / kUT) * kUT;  // multiple of the 128-token step
   const size_t snap_head = (size_t)nsnap * 65 * m_pad * 2;
-  const size_t kt_head = (size_t)65 * Npad * 2;
-  const size_t per_head = snap_head + kt_head;
+  const size_t kt_head = (size_t)65 * Npad * 2;  // K^T or V^T of one head
+  const size_t per_head = snap_head + 2 * kt_head;
   const size_t budget = (size_t)4 << 30;
   const int G = (int)std::max<size_t>(1, std::min<size_t>(BH, budget / per_head));
   int st = SATA_OK;
-  uint8_t *ws = (uint8_t *)get_workspace(stream, per_head * G + 256, &st);
+  uint8_t *ws = (uint8_t *)get_workspace(stream, per_head * G + 1024, &st);
   if (!ws) return st;
+  const size_t kt_bytes = (kt_head * G + 255) & ~(size_t)255;
   __nv_bfloat16 *kt = reinterpret_cast<__nv_bfloat16 *>(ws);
-  __nv_bfloat16 *snap =
-      reinterpret_cast<__nv_bfloat16 *>(ws + ((kt_head * G + 255) & ~(size_t)255));
-  CUtensorMap mV64, mVU, mQ, mK64, mS, mKT;
+  __nv_bfloat16 *vt = reinterpret_cast<__nv_bfloat16 *>(ws + kt_bytes);
+  __nv_bfloat16 *snap = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * kt_bytes);
+  CUtensorMap mV64, mQ, mK64, mS, mKT, mVT;
   if (!make_map(&mV64, v, 64, N, BH, 64) || !make_map(&mK64, k, 64, N, BH, 64) ||
-      !make_map(&mVU, v, 64, N, BH, kUT) || !make_map(&mQ, q, 64, N, BH, 128))
+      !make_map(&mQ, q, 64, N, BH, 128))
     return SATA_ERR_CUDA;
   static bool attr_done = false;
   if (!attr_done) {
@@ -720,12 +726,15 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
   ones.w3 = ones.w3h = ones.w3s = ones.w2 = ones.w2h = ones.w1 = 1.f;
   for (int h0 = 0; h0 < BH; h0 += G) {
     const int g = std::min(G, BH - h0);
-    if (!make_map(&mKT, kt, (uint64_t)Npad, 65, (uint64_t)g, 65)) return SATA_ERR_CUDA;
+    if (!make_map(&mKT, kt, (uint64_t)Npad, 65, (uint64_t)g, 65) ||
+        !make_map(&mVT, vt, (uint64_t)Npad, 65, (uint64_t)g, kNP))
+      return SATA_ERR_CUDA;
     if (nsnap > 0 && !make_map(&mS, snap, (uint64_t)m_pad, 65, (uint64_t)g * nsnap, kNP))
       return SATA_ERR_CUDA;
     prof_kernel_begin(stream, K_TC_PREP);
-    tc_transpose_k<<<dim3(Npad / 64, g), 256, 0, stream>>>(
-        reinterpret_cast<const __nv_bfloat16 *>(k), kt, N, Npad, h0);
+    tc_transpose_kv<<<dim3(Npad / 64, g), 256, 0, stream>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(k), reinterpret_cast<const __nv_bfloat16 *>(v),
+        kt, vt, N, Npad, h0);
     prof_kernel_end(stream);
     UParams up;
     up.slot_idx = basis->slot_idx;
@@ -744,7 +753,7 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
     up.state = state;
     up.err = err;
     prof_kernel_begin(stream, K_TC_CHUNK_STATES);
-    tc_chunk_states<<<std::min(up.n_items, nsm), kUThreads, kUSmem, stream>>>(mKT, mVU, up);
+    tc_chunk_states<<<std::min(up.n_items, nsm), kUThreads, kUSmem, stream>>>(mKT, mVT, up);
     prof_kernel_end(stream);
     RParams rp;
     rp.tiles = reinterpret_cast<const TileDesc *>(basis->tile_desc);
