@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
   uint8_t *sKT = smem + kUOffKT, *sVT = smem + kUOffVT;
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kUOffBar);
   uint64_t *kv_full = bar, *kv_empty = bar + kUKS, *a_full = bar + 2 * kUKS,
-           *a_empty = a_full + kUAS, *snap_full = a_empty + kUAS, *snap_done = snap_full + 1,
+           *a_empty = a_full + kUAS, *snap_full = a_empty + kUAS, *snap_done = snap_full + kUF,
            *drain = snap_done + kUF;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(drain + 2);
@@ -124,8 +124,10 @@ __global__ void __launch_bounds__(kUThreads, 1)
       mbar_init(&a_full[s], kUGenWarps);
       mbar_init(&a_empty[s], 1);
     }
-    mbar_init(snap_full, 1);
-    for (int f = 0; f < kUF; ++f) mbar_init(&snap_done[f], 4);
+    for (int f = 0; f < kUF; ++f) {
+      mbar_init(&snap_full[f], 1);
+      mbar_init(&snap_done[f], 4);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -184,6 +186,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
           if (!(ok = mbar_wait(&a_full[as], (it / kUAS) & 1, abort_flag, p.err))) break;
           tc_fence_after();
           const uint32_t b0 = smem_u32(sVT + ks * kUVT);
+          const bool event = is_event(s);
           for (int f = 0; f < kUF; ++f) {
             // every tile's barrier is waited once per event, in order, so no
             // barrier can run two phases ahead of its waiter
@@ -198,13 +201,16 @@ __global__ void __launch_bounds__(kUThreads, 1)
               const uint64_t bd = smem_desc_sw128(b0 + (k >> 2) * kUVTh + 32 * (k & 3), 16, 1024);
               mma_bf16_ts(tmem + f * kNP, a0 + 8 * k, bd, idesc, (s > 0 || k > 0) ? 1u : 0u);
             }
+            // tile f's snapshot can leave TMEM as soon as its own MMAs are done,
+            // while the tensor core continues with the next tile
+            if (event) mma_commit(&snap_full[f]);
           }
           if (!ok) break;
           after_event = false;
           mma_commit(&a_empty[as]);
           mma_commit(&kv_empty[ks]);
-          if (is_event(s)) {
-            mma_commit(snap_full);
+          if (event) {
+            for (int f = nmt; f < kUF; ++f) mma_commit(&snap_full[f]);  // absent tiles
             ++events;
             after_event = true;
           }
@@ -225,12 +231,11 @@ __global__ void __launch_bounds__(kUThreads, 1)
       const int hb = item / p.n_batches, batch = item % p.n_batches;
       for (int s = 0; ok && s < nsub; ++s) {
         if (!is_event(s)) continue;
-        if (!(ok = mbar_wait(snap_full, events & 1, abort_flag, p.err))) break;
-        ++events;
-        tc_fence_after();
         const bool boundary = s != nsub - 1;
         const int c = boundary ? (s + 1) / sub_per_chunk - 1 : 0;
-        for (int f = 0; f < kUF; ++f) {
+        for (int f = 0; ok && f < kUF; ++f) {
+          if (!(ok = mbar_wait(&snap_full[f], events & 1, abort_flag, p.err))) break;
+          tc_fence_after();
           const int mt = batch * kUF + f;
           const bool live = mt < p.n_mt;
           const int slot = mt * 128 + row;
@@ -259,6 +264,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
             for (int n = 0; n < 65; ++n) tdst[n] = scale * __uint_as_float(v[n]);
           }
         }
+        ++events;
       }
     }
   } else {
@@ -536,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&a_empty[st]);
           mma_commit(&b_empty[bs]);
-          intra(false);
+          if (i & 1) intra(false);
         }
       }
       if (ok) intra(true);
