@@ -215,6 +215,32 @@ def cpu_baseline(budget_s: float = 20.0):
                                  f"{ddt:.2f} s"}}
 
 
+# --------------------------------------------------------------- ranks
+def dist_barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def dist_max(x: float, world: int, device=None) -> float:
+    """Max of x over all ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, steps: int, units_per_step_per_rank: float,
+                       max_total_ms: float) -> float:
+    """Whole-job throughput: every rank processes its own units each step."""
+    return world * steps * units_per_step_per_rank / (max_total_ms / 1e3)
+
+
 # --------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import numpy as np
@@ -229,19 +255,10 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
 
     def barrier():
-        if world > 1:
-            import torch.distributed as dist
-
-            dist.barrier()
+        dist_barrier(world)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        import torch.distributed as dist
-
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return dist_max(x, world, dev)
 
     vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
     phys = vis[local_rank] if local_rank < len(vis) else str(local_rank)
@@ -286,7 +303,7 @@ def run_ours(args, rank, world, local_rank):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = max_over_ranks(sum(step_ms))
     prefill_tokens = w["B"] * w["N"]
-    value = world * args.steps * prefill_tokens / (total_ms / 1e3)
+    value = weak_scaling_value(world, args.steps, prefill_tokens, total_ms)
     assert sata.sata_get_error() == sata.SATA_OK
 
     # dominant kernel of the prefill step
@@ -330,7 +347,8 @@ def run_ours(args, rank, world, local_rank):
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
     e2e_total = max_over_ranks(sum(e2e_ms))
-    e2e = {"value": world * args.steps * prefill_tokens / (e2e_total / 1e3), "unit": "tokens/s",
+    e2e = {"value": weak_scaling_value(world, args.steps, prefill_tokens, e2e_total),
+           "unit": "tokens/s",
            "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (q, k, v)),
            "d2h_bytes_per_step": out.numel() * 4 + state.numel() * 4}
     del qd, kd, vd, out, state, q, k, v, qh, kh, vh, out_h, st_h
@@ -376,7 +394,7 @@ def run_ours(args, rank, world, local_rank):
     sata.sata_profile_enable(False)
     dms = [a.elapsed_time(b) for a, b in dev_ev]
     dtotal = max_over_ranks(sum(dms))
-    dvalue = world * nsteps * dw["B"] / (dtotal / 1e3)
+    dvalue = weak_scaling_value(world, nsteps, dw["B"], dtotal)
     dbytes = 2 * dw["B"] * dw["H"] * dm * (dw["dV"] + 1) * 4
     dkern_ms = statistics.mean(dk["decode_stream"])
     dach = dbytes / (dkern_ms / 1e3) / 1e9
