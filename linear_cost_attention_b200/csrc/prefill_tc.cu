@@ -182,7 +182,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
         const int nmt = min(kUF, p.n_mt - batch * kUF);
         for (int s = 0; ok && s < nsub; ++s, ++it) {
           const int ks = it % kUKS, as = it % kUAS;
-          if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err))) break;
+          // a_full also covers kv_full: every generator warp waited on kv_full[ks]
+          // before arriving.  One barrier wait per step: a wait in this thread
+          // stalls until the MMAs already issued have drained.
           if (!(ok = mbar_wait(&a_full[as], (it / kUAS) & 1, abort_flag, p.err))) break;
           tc_fence_after();
           const uint32_t b0 = smem_u32(sVT + ks * kUVT);
@@ -351,9 +353,9 @@ __global__ void __launch_bounds__(256) tc_transpose_kv(const __nv_bfloat16 *__re
 }
 
 // ============================================================ readout
-constexpr int kRTS = 3;                  // feature tiles per pipeline stage
-constexpr int kRStages = 3;              // phi(Q) stages, in TMEM (32 columns per tile)
-constexpr int kRBS = 4;                  // snapshot stages (kRTS tiles each)
+constexpr int kRTS = 4;                  // feature tiles per pipeline stage
+constexpr int kRStages = 2;              // phi(Q) stages, in TMEM (32 columns per tile)
+constexpr int kRBS = 3;                  // snapshot stages (kRTS tiles each)
 constexpr int kKB = 64;                  // keys per in-chunk block
 constexpr uint32_t kRTile = 128 * kRow;  // 128 tokens x 64 features: 16 KiB
 constexpr uint32_t kRB = kNP * kRow;     // 80 x 64 snapshot tile: 10 KiB
@@ -528,8 +530,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n_stages = (p.n_tiles + kRTS - 1) / kRTS;
         for (int i = 0; i < n_stages; ++i) {
           const int st = i % kRStages, bs = i % kRBS;
+          // a_full also covers b_full: the generator warps wait on the snapshot
+          // stage before arriving (one barrier wait per stage in this thread)
           if (!(ok = mbar_wait(&a_full[st], (i / kRStages) & 1, abort_flag, p.err))) break;
-          if (!(ok = mbar_wait(&b_full[bs], (i / kRBS) & 1, abort_flag, p.err))) break;
           tc_fence_after();
           const int nt = min(kRTS, p.n_tiles - kRTS * i);
           for (int t = 0; t < nt; ++t) {
@@ -635,6 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st32(tmem + ((uint32_t)(32 * (gw & 3)) << 16) + kRColA + (st * kRTS + t) * 32, out);
       }
       tmem_st_wait();
+      if (!(ok = mbar_wait(&b_full[i % kRBS], (i / kRBS) & 1, abort_flag, p.err))) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&a_full[st]);
