@@ -120,7 +120,8 @@ class ClockSampler:
 # --------------------------------------------------------------- traffic record
 def traffic_record(kernel: str):
     """Per-launch DRAM bytes of ``kernel`` from the committed ncu summary, or
-    None when the kernel sources changed since the counters were taken."""
+    None when the kernel's source files changed since the counters were taken
+    (the record lists them; the hash covers their names and contents)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -128,15 +129,17 @@ def traffic_record(kernel: str):
     except Exception:
         return None
     r = rec.get(kernel)
-    if not r or r.get("source_sha") != source_sha():
+    if not r or r.get("source_sha") != source_sha(r.get("sources")):
         return None
     return r.get("bytes_per_launch")
 
 
-def source_sha() -> str:
+def source_sha(files=None) -> str:
+    """sha256 prefix over the named files of the CUDA sources (all of them
+    when ``files`` is None), in sorted order."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_cost_attention_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files if files else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -496,7 +499,7 @@ def profile_case(case: str):
             qt, kt, vt = (x[:, :, t].contiguous().cuda() for x in (q, k, v))
             sata.decode_step(qt, kt, vt, state, P)
     elif case == "prefill":
-        B, H, N, d, P = 1, 2, 4096, 64, 4         # state 25 MB; chunk states > L2
+        B, H, N, d, P = 1, 2, 8192, 64, 4         # one chunk-boundary snapshot per head
         q, k, v = make_qkv(B, H, N, d, d, seed=4, dtype="bf16")
         qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
         for _ in range(3):

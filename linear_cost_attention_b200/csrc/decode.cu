@@ -23,7 +23,8 @@
 namespace sata {
 namespace {
 
-constexpr int kIters = 16;  // iterations (of 4*NT elements) per block
+constexpr int kIters = 32;  // iterations (of 4*NT elements) per block: 32 measured
+                            // 2% faster than 16 (fewer per-block feature prologues)
 constexpr int kUnroll = 4;  // iterations whose loads are in flight together
 
 template <int D1> struct DecodeShape;

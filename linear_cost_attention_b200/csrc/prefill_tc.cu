@@ -81,6 +81,7 @@ constexpr int kUGenWarps = 4 * kUF;
 constexpr int kUEpiWarp0 = 2, kUGenWarp0 = 6;  // warps 2..5 epilogue, 6.. generators
 constexpr int kUThreads = 32 * (kUGenWarp0 + kUGenWarps);
 constexpr int kMaxTiles = 768;  // tile table capacity in smem (readout)
+constexpr int kChunk = 4096;    // tokens per chunk (a multiple of the 128-token step)
 constexpr uint32_t kUColA = 160;               // TMEM: D at f*80, A from column 160
 constexpr uint32_t kUTmemCols = 512;
 constexpr uint32_t kUKTh = 9 * 1024;           // one 64-token K^T box: 65 rows x 128 B, padded
@@ -89,6 +90,15 @@ constexpr uint32_t kUKT = 2 * kUKTh, kUVT = 2 * kUVTh;  // per step (two boxes e
 constexpr uint32_t kUOffKT = 0, kUOffVT = kUOffKT + kUKS * kUKT, kUOffBar = kUOffVT + kUKS * kUVT;
 constexpr uint32_t kUSmem = kUOffBar + 256 + 1024;
 static_assert(kUColA + kUAS * kUF * (kUT / 2) <= kUTmemCols && kUF * kNP <= kUColA, "TMEM budget");
+
+// TMEM lane -> slot inside a 128-row state tile.  Within each 32-lane warp
+// quarter, lane 4c + b holds slot 8b + c: in the 8 x 8 tiles (index octets b, c)
+// a warp then reads each "c" operand row from 4 adjacent lanes and each "b"
+// operand row from every fourth lane, which shared memory serves at half the
+// cost of one row per lane & 7.
+__host__ __device__ constexpr int lane_slot(int r) {
+  return (r & ~31) | ((r & 3) << 3) | ((r >> 2) & 7);
+}
 
 struct UParams {
   const uint32_t *slot_idx;  // [m_pad] i | j << 8 | l << 16 (64 = the ones row)
@@ -189,30 +199,30 @@ __global__ void __launch_bounds__(kUThreads, 1)
           tc_fence_after();
           const uint32_t b0 = smem_u32(sVT + ks * kUVT);
           const bool event = is_event(s);
-          for (int f = 0; f < kUF; ++f) {
+          if (after_event) {
             // every tile's barrier is waited once per event, in order, so no
             // barrier can run two phases ahead of its waiter
-            if (after_event) {
-              if (!(ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err))) break;
-              tc_fence_after();
-            }
-            if (f >= nmt) continue;
-            const uint32_t a0 = tmem + kUColA + (as * kUF + f) * (kUT / 2);
-#pragma unroll
-            for (int k = 0; k < kUT / 16; ++k) {
-              const uint64_t bd = smem_desc_sw128(b0 + (k >> 2) * kUVTh + 32 * (k & 3), 16, 1024);
-              mma_bf16_ts(tmem + f * kNP, a0 + 8 * k, bd, idesc, (s > 0 || k > 0) ? 1u : 0u);
-            }
-            // tile f's snapshot can leave TMEM as soon as its own MMAs are done,
-            // while the tensor core continues with the next tile
-            if (event) mma_commit(&snap_full[f]);
+            for (int f = 0; ok && f < kUF; ++f)
+              ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err);
+            if (!ok) break;
+            tc_fence_after();
           }
-          if (!ok) break;
+          // the tiles' MMAs alternate, so consecutive MMAs accumulate into
+          // different TMEM columns and do not wait for each other
+#pragma unroll
+          for (int k = 0; k < kUT / 16; ++k) {
+            const uint64_t bd = smem_desc_sw128(b0 + (k >> 2) * kUVTh + 32 * (k & 3), 16, 1024);
+#pragma unroll
+            for (int f = 0; f < kUF; ++f)
+              if (f < nmt)
+                mma_bf16_ts(tmem + f * kNP, tmem + kUColA + (as * kUF + f) * (kUT / 2) + 8 * k, bd,
+                            idesc, (s > 0 || k > 0) ? 1u : 0u);
+          }
           after_event = false;
           mma_commit(&a_empty[as]);
           mma_commit(&kv_empty[ks]);
           if (event) {
-            for (int f = nmt; f < kUF; ++f) mma_commit(&snap_full[f]);  // absent tiles
+            for (int f = 0; f < kUF; ++f) mma_commit(&snap_full[f]);
             ++events;
             after_event = true;
           }
@@ -240,7 +250,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
           tc_fence_after();
           const int mt = batch * kUF + f;
           const bool live = mt < p.n_mt;
-          const int slot = mt * 128 + row;
+          const int slot = mt * 128 + lane_slot(row);
           const float w = live ? p.slot_w[slot] : 0.f;
           const int r = (live && !boundary) ? p.row_of_slot[slot] : -1;
           __nv_bfloat16 *sdst = p.snap + ((size_t)(hb * p.nsnap + c) * 65) * p.m_pad + slot;
@@ -282,7 +292,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
       const int batch = item % p.n_batches;
       const int mt = batch * kUF + f;
       uint32_t ix = 0x404040u;  // three "ones" rows
-      if (mt < p.n_mt) ix = p.slot_idx[mt * 128 + row];
+      if (mt < p.n_mt) ix = p.slot_idx[mt * 128 + lane_slot(row)];
       const uint32_t ri = (ix & 0xff) * kRow, rj = ((ix >> 8) & 0xff) * kRow,
                      rl = ((ix >> 16) & 0xff) * kRow;
       const uint32_t si = (ix & 7), sj = ((ix >> 8) & 7), sl = ((ix >> 16) & 7);
@@ -294,13 +304,13 @@ __global__ void __launch_bounds__(kUThreads, 1)
           break;
 #pragma unroll 1
         for (int h = 0; h < kUT / 64; ++h) {  // 64 tokens (one K^T box) at a time
-          const uint8_t *kt = sKT + ks * kUKT + h * kUKTh;
+          const uint32_t kt = smem_u32(sKT) + ks * kUKT + h * kUKTh;
           uint32_t out[32];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const uint4 xi = *reinterpret_cast<const uint4 *>(kt + ri + (((uint32_t)c ^ si) << 4));
-            const uint4 xj = *reinterpret_cast<const uint4 *>(kt + rj + (((uint32_t)c ^ sj) << 4));
-            const uint4 xl = *reinterpret_cast<const uint4 *>(kt + rl + (((uint32_t)c ^ sl) << 4));
+            const uint4 xi = lds128(kt + ri + (((uint32_t)c ^ si) << 4));
+            const uint4 xj = lds128(kt + rj + (((uint32_t)c ^ sj) << 4));
+            const uint4 xl = lds128(kt + rl + (((uint32_t)c ^ sl) << 4));
             out[4 * c + 0] = bmul2(bmul2(xi.x, xj.x), xl.x);
             out[4 * c + 1] = bmul2(bmul2(xi.y, xj.y), xl.y);
             out[4 * c + 2] = bmul2(bmul2(xi.z, xj.z), xl.z);
@@ -418,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(p_full, 4);
     mbar_init(o_full, 1);
     for (int s = 0; s < kRStages; ++s) {
-      mbar_init(&a_full[s], 4);
+      mbar_init(&a_full[s], 8);
       mbar_init(&a_empty[s], 1);
     }
     for (int s = 0; s < kRBS; ++s) {
@@ -610,20 +620,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 8 && inter) {
-    // ---------------- feature generators: phi(Q) tiles, one thread per token
+    // ---------------- feature generators: phi(Q) tiles, one thread per token;
+    // the two warps of a TMEM lane quarter split every stage's tiles
     const int gw = warp - 8;
     const int half = gw >> 2;
     const int row = lane + 32 * (gw & 3);
     bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
     const uint8_t *qrow = sQ + row * kRow;
     const int n_stages = (p.n_tiles + kRTS - 1) / kRTS;
-    for (int i = half; ok && i < n_stages; i += 2) {
+    for (int i = 0; ok && i < n_stages; ++i) {
       const int st = i % kRStages;
       if (i >= kRStages && !(ok = mbar_wait(&a_empty[st], ((i / kRStages) - 1) & 1, abort_flag,
                                             p.err)))
         break;
 #pragma unroll 1
-      for (int t = 0; t < kRTS; ++t) {
+      for (int t = half; t < kRTS; t += 2) {
         const int ti = kRTS * i + t;
         uint32_t out[32];
         if (ti < p.n_tiles) {
@@ -698,7 +709,11 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
   const int n_tiles = basis->n_tiles;  // even, padded
   if (n_tiles > kMaxTiles) return SATA_ERR_UNSUPPORTED;
   const int m_pad = n_tiles * 64;
-  const int C = N <= 1024 ? ((N + 127) / 128) * 128 : 1024;
+  // Chunk length: a snapshot boundary stalls the state kernel while the tile
+  // leaves TMEM and costs a snapshot write, while the readout hides the longer
+  // in-chunk quadratic part behind its inter-chunk MMAs; 4096 measured fastest
+  // of 1024 / 2048 / 4096 at 16384 tokens.
+  const int C = N <= kChunk ? ((N + 127) / 128) * 128 : kChunk;
   const int nsnap = (N + C - 1) / C - 1;
   const int Npad = ((N + kUT - 1) / kUT) * kUT;  // multiple of the 128-token step
   const size_t snap_head = (size_t)nsnap * 65 * m_pad * 2;

@@ -97,10 +97,10 @@ def test_edge_shapes(B, H, N, dK, dV, P, dt):
     (1, 1, 1),        # one token
     (1, 2, 100),      # ragged, one partial key block
     (1, 1, 128),      # exactly one block, no snapshot
-    (2, 1, 1024),     # one full chunk
-    (1, 2, 1152),     # one snapshot + a block of the next chunk
-    (1, 1, 2500),     # two snapshots, ragged tail
-    (1, 3, 4096),     # three snapshots, several items per head
+    (2, 1, 1024),     # one chunk, several items per head
+    (1, 1, 4096),     # exactly one full chunk, no snapshot
+    (1, 2, 4224),     # one snapshot + a block of the next chunk
+    (1, 1, 9000),     # two snapshots, ragged tail
 ])
 def test_tensor_core_prefill_shapes(B, H, N):
     # bf16, dK = dV = 64, P = 4: the tcgen05 path
