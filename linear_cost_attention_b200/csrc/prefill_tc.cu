@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kUKS; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1 + kUGenWarps);
+      mbar_init(&kv_empty[s], kUGenWarps);
     }
     for (int s = 0; s < kUAS; ++s) {
       mbar_init(&a_full[s], kUGenWarps);
@@ -219,8 +219,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
                             idesc, (s > 0 || k > 0) ? 1u : 0u);
           }
           after_event = false;
+          // one commit per step: the generators release the K^T / V^T stage
+          // once this commit has fired (each tcgen05.commit costs pipe time)
           mma_commit(&a_empty[as]);
-          mma_commit(&kv_empty[ks]);
           if (event) {
             for (int f = 0; f < kUF; ++f) mma_commit(&snap_full[f]);
             ++events;
@@ -299,9 +300,13 @@ __global__ void __launch_bounds__(kUThreads, 1)
       for (int s = 0; ok && s < nsub; ++s, ++it) {
         const int ks = it % kUKS, as = it % kUAS;
         if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err))) break;
-        if (it >= kUAS &&
-            !(ok = mbar_wait(&a_empty[as], ((it / kUAS) - 1) & 1, abort_flag, p.err)))
-          break;
+        if (it >= kUAS) {
+          if (!(ok = mbar_wait(&a_empty[as], ((it / kUAS) - 1) & 1, abort_flag, p.err))) break;
+          // the MMAs of step it - kUAS are complete and this warp read its K^T
+          // rows long ago: release that step's K^T / V^T stage
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&kv_empty[(it - kUAS) % kUKS]);
+        }
 #pragma unroll 1
         for (int h = 0; h < kUT / 64; ++h) {  // 64 tokens (one K^T box) at a time
           const uint32_t kt = smem_u32(sKT) + ks * kUKT + h * kUKTh;
@@ -321,10 +326,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&a_full[as]);
-          mbar_arrive(&kv_empty[ks]);
-        }
+        if (lane == 0) mbar_arrive(&a_full[as]);
       }
     }
   }
