@@ -89,6 +89,25 @@ int sata_prefill(const void *q, const void *k, const void *v, float *out,
                  float *state, int B, int H, int N, int dK, int dV, int P,
                  sata_dtype dt, sata_stream_t stream);
 
+/* Causal prefill that continues from an existing state (a prompt continued
+ * in pieces, or chunked prefill): "恒定计算成本的工程实现" folds every token into
+ * the fixed-size state, so the tokens before this call enter only through
+ * S_0, the state after them (as written by sata_prefill, sata_prefill_continue
+ * or sata_decode_step).  Same arguments and layouts as sata_prefill, except
+ * that `state` is read as S_0 and then overwritten with the state after these
+ * N tokens; out_i = (phi(q_i)^T (S_0 + sum_{j<=i} phi(k_j)[v_j,1]^T)) read
+ * and normalised as in sata_prefill (j over this call's tokens, inclusive).
+ * With S_0 = 0 the result equals sata_prefill's; prefill of N_0 tokens then
+ * continuing with N_1 tokens gives the outputs of tokens N_0.. and the state
+ * of one prefill of N_0 + N_1 tokens, up to rounding (on the tensor-core path
+ * S_0 enters the readout rounded to bf16, like every chunk-boundary state).
+ * Returns SATA_OK, SATA_ERR_INVALID_ARG, SATA_ERR_UNSUPPORTED, SATA_ERR_NOMEM
+ * or SATA_ERR_CUDA. */
+int sata_prefill_continue(const void *q, const void *k, const void *v,
+                          float *out, float *state, int B, int H, int N,
+                          int dK, int dV, int P, sata_dtype dt,
+                          sata_stream_t stream);
+
 /* One single-token step for each of B*H heads ("恒定计算成本的工程实现":
  * per-token procedure at constant cost): state += phi(k) [v, 1]^T in place,
  * then out = (phi(q)^T state)[:dV] / (phi(q)^T state)[dV].  The token attends

@@ -54,6 +54,8 @@ def lib() -> ctypes.CDLL:
     L.sata_index_table.restype = i64
     L.sata_prefill.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
     L.sata_prefill.restype = i
+    L.sata_prefill_continue.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    L.sata_prefill_continue.restype = i
     L.sata_decode_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     L.sata_decode_step.restype = i
     L.sata_get_error.argtypes = [vp]
@@ -126,6 +128,13 @@ def sata_prefill(q, k, v, out, state, B, H, N, dK, dV, P, dtype, stream=None) ->
                             dV, P, _dtype_code(dtype), _stream(stream))
     if st != SATA_OK:
         raise SataError(st, "sata_prefill")
+
+
+def sata_prefill_continue(q, k, v, out, state, B, H, N, dK, dV, P, dtype, stream=None) -> None:
+    st = lib().sata_prefill_continue(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state), B, H,
+                                     N, dK, dV, P, _dtype_code(dtype), _stream(stream))
+    if st != SATA_OK:
+        raise SataError(st, "sata_prefill_continue")
 
 
 def sata_decode_step(q, k, v, state, out, B, H, dK, dV, P, dtype, stream=None) -> None:
@@ -201,6 +210,21 @@ def prefill(q, k, v, P: int, out=None, state=None, stream=None):
         state = torch.empty(B, H, m, dV + 1, device=q.device, dtype=torch.float32)
     sata_prefill(q, k, v, out, state, B, H, N, dK, dV, P, q.dtype, stream)
     return out, state
+
+
+def prefill_continue(q, k, v, state, P: int, out=None, stream=None):
+    """Causal prefill continuing from ``state`` (the state after earlier
+    tokens, [B,H,m,dV+1] fp32, updated in place): q,k [B,H,N,dK], v [B,H,N,dV]
+    -> out [B,H,N,dV] fp32."""
+    import torch
+
+    _check_qkv(q, k, v)
+    B, H, N, dK = q.shape
+    dV = v.shape[-1]
+    if out is None:
+        out = torch.empty(B, H, N, dV, device=q.device, dtype=torch.float32)
+    sata_prefill_continue(q, k, v, out, state, B, H, N, dK, dV, P, q.dtype, stream)
+    return out
 
 
 def decode_step(q, k, v, state, P: int, out=None, stream=None):

@@ -9,6 +9,9 @@
 //   kernel 2 (readout): for a block of tokens in chunk c,
 //     [num, den]_i = phi(q_i)^T S_(before c)  +  sum_{c0 <= j <= i} T_P(s_ij) [v_j, 1]
 //     and out_i = num_i / den_i.
+// A continued prefill starts kernel 1 from the caller's state S_0 instead of
+// zero and stores S_0 as the state before chunk 0 (snapshot slot 0); the
+// snapshot before chunk c then sits in slot c instead of c - 1.
 // Both terms are exact reorganisations of sum_{j<=i} T_P(s_ij)[v_j,1]
 // ("对称张量分解的核心洞察": phi(q).phi(k) = T_P(q.k/sqrt(dK)) over the minimal
 // basis), so the result equals the quadratic form up to rounding.
@@ -30,7 +33,7 @@ __global__ void __launch_bounds__(kThreads)
     simt_chunk_states(const T *__restrict__ k, const T *__restrict__ v,
                       const uint32_t *__restrict__ idx, const float *__restrict__ w,
                       int m, int N, int C, int head0, float *__restrict__ snap, int nsnap,
-                      float *__restrict__ state) {
+                      int cont, float *__restrict__ state) {
   constexpr int D1 = DV + 1;
   constexpr int ENT = kFT * D1;
   constexpr int R = (ENT + kThreads - 1) / kThreads;
@@ -49,14 +52,21 @@ __global__ void __launch_bounds__(kThreads)
     sw[tid] = a < m ? w[a] : 0.f;
   }
   float acc[R];
+  float *st = state + bh * (size_t)m * D1;
 #pragma unroll
-  for (int r = 0; r < R; ++r) acc[r] = 0.f;
+  for (int r = 0; r < R; ++r) {
+    // a continued prefill starts from the caller's state (read here, by the
+    // thread that overwrites the same entries at the end)
+    const int e = tid + r * kThreads;
+    acc[r] = 0.f;
+    if (cont && e < ENT && a0 + e / D1 < m) acc[r] = st[(size_t)(a0 + e / D1) * D1 + e % D1];
+  }
   const T *kh = k + bh * N * DK;
   const T *vh = v + bh * N * DV;
 
   for (int t0 = 0; t0 < N; t0 += kTT) {
-    if (t0 > 0 && t0 % C == 0) {
-      float *sp = snap + ((size_t)blockIdx.y * nsnap + (t0 / C - 1)) * (size_t)m * D1;
+    if ((t0 > 0 || cont) && t0 % C == 0) {
+      float *sp = snap + ((size_t)blockIdx.y * nsnap + (t0 / C - 1 + cont)) * (size_t)m * D1;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         const int e = tid + r * kThreads;
@@ -97,7 +107,6 @@ __global__ void __launch_bounds__(kThreads)
       }
     }
   }
-  float *st = state + bh * (size_t)m * D1;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const int e = tid + r * kThreads;
@@ -113,7 +122,7 @@ __global__ void __launch_bounds__(kThreads)
     simt_readout(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                  const uint32_t *__restrict__ idx, const float *__restrict__ w, int m, int N,
                  int C, int P, int head0, const float *__restrict__ snap, int nsnap,
-                 float *__restrict__ out) {
+                 int cont, float *__restrict__ out) {
   static_assert(kTB == kFT && kTB == kTT, "tile sizes share shared-memory buffers");
   constexpr int D1 = DV + 1;
   constexpr int ENT = kTB * D1;
@@ -146,8 +155,8 @@ __global__ void __launch_bounds__(kThreads)
   for (int r = 0; r < R; ++r) acc[r] = 0.f;
 
   // inter-chunk: phi(q_i)^T S_(before chunk)
-  if (chunk > 0) {
-    const float *sp = snap + ((size_t)blockIdx.y * nsnap + (chunk - 1)) * (size_t)m * D1;
+  if (chunk > 0 || cont) {
+    const float *sp = snap + ((size_t)blockIdx.y * nsnap + (chunk - 1 + cont)) * (size_t)m * D1;
     for (int a0 = 0; a0 < m; a0 += kFT) {
       __syncthreads();
       if (tid < kFT) {
@@ -235,13 +244,13 @@ __global__ void __launch_bounds__(kThreads)
 
 template <int DK, int DV, typename T>
 int run_simt(const void *q, const void *k, const void *v, float *out, float *state, int BH,
-             int N, int P, const DeviceBasis *basis, cudaStream_t stream) {
+             int N, int P, bool cont, const DeviceBasis *basis, cudaStream_t stream) {
   const int m = (int)basis->m;
   constexpr int D1 = DV + 1;
   // Chunk length: a multiple of 64 giving at most 16 chunks.
   const int C = std::max(64, ((N + 16 * 64 - 1) / (16 * 64)) * 64);
   const int nchunks = (N + C - 1) / C;
-  const int nsnap = nchunks - 1;
+  const int nsnap = nchunks - 1 + (cont ? 1 : 0);  // + slot 0 = initial state
   const size_t per_head = (size_t)std::max(nsnap, 0) * m * D1 * sizeof(float);
   const size_t budget = (size_t)1 << 30;
   int G = BH;
@@ -258,12 +267,14 @@ int run_simt(const void *q, const void *k, const void *v, float *out, float *sta
     dim3 g1((m + kFT - 1) / kFT, g);
     prof_kernel_begin(stream, K_SIMT_CHUNK_STATES);
     simt_chunk_states<DK, DV, T><<<g1, kThreads, 0, stream>>>(kk, vv, basis->idx, basis->w, m, N,
-                                                               C, h0, snap, nsnap, state);
+                                                               C, h0, snap, nsnap, cont ? 1 : 0,
+                                                               state);
     prof_kernel_end(stream);
     dim3 g2((N + kTB - 1) / kTB, g);
     prof_kernel_begin(stream, K_SIMT_READOUT);
     simt_readout<DK, DV, T><<<g2, kThreads, 0, stream>>>(qq, kk, vv, basis->idx, basis->w, m, N,
-                                                          C, P, h0, snap, nsnap, out);
+                                                          C, P, h0, snap, nsnap, cont ? 1 : 0,
+                                                          out);
     prof_kernel_end(stream);
   }
   return cuda_status(cudaGetLastError());
@@ -271,9 +282,11 @@ int run_simt(const void *q, const void *k, const void *v, float *out, float *sta
 
 template <typename T>
 int dispatch_dv(int dK, int dV, const void *q, const void *k, const void *v, float *out,
-                float *state, int BH, int N, int P, const DeviceBasis *b, cudaStream_t s) {
-#define SATA_CASE(DKV, DVV) \
-  if (dK == DKV && dV == DVV) return run_simt<DKV, DVV, T>(q, k, v, out, state, BH, N, P, b, s);
+                float *state, int BH, int N, int P, bool cont, const DeviceBasis *b,
+                cudaStream_t s) {
+#define SATA_CASE(DKV, DVV)        \
+  if (dK == DKV && dV == DVV)      \
+    return run_simt<DKV, DVV, T>(q, k, v, out, state, BH, N, P, cont, b, s);
 #define SATA_ROW(DKV) SATA_CASE(DKV, 8) SATA_CASE(DKV, 16) SATA_CASE(DKV, 32) SATA_CASE(DKV, 64)
   SATA_ROW(8) SATA_ROW(16) SATA_ROW(32) SATA_ROW(64)
 #undef SATA_ROW
@@ -284,12 +297,13 @@ int dispatch_dv(int dK, int dV, const void *q, const void *k, const void *v, flo
 }  // namespace
 
 int launch_prefill_simt(const void *q, const void *k, const void *v, float *out, float *state,
-                        int B, int H, int N, int dK, int dV, int P, bool bf16,
+                        int B, int H, int N, int dK, int dV, int P, bool bf16, bool cont,
                         const DeviceBasis *basis, cudaStream_t stream) {
   const int BH = B * H;
   if (bf16)
-    return dispatch_dv<__nv_bfloat16>(dK, dV, q, k, v, out, state, BH, N, P, basis, stream);
-  return dispatch_dv<float>(dK, dV, q, k, v, out, state, BH, N, P, basis, stream);
+    return dispatch_dv<__nv_bfloat16>(dK, dV, q, k, v, out, state, BH, N, P, cont, basis,
+                                      stream);
+  return dispatch_dv<float>(dK, dV, q, k, v, out, state, BH, N, P, cont, basis, stream);
 }
 
 }  // namespace sata

@@ -106,7 +106,8 @@ struct UParams {
   const int32_t *row_of_slot;
   int n_mt;                  // 128-row tiles (m_pad / 128)
   int N, C, nsnap, m, m_pad, n_batches, n_items, head0;
-  __nv_bfloat16 *snap;  // [G][nsnap][65][m_pad]
+  int cont;             // 1: start from the state in `state` (continued prefill)
+  __nv_bfloat16 *snap;  // [G][nsnap][65][m_pad]; slot 0 = initial state if cont
   float *state;         // [BH][m][65]
   int *err;
 };
@@ -120,9 +121,10 @@ __global__ void __launch_bounds__(kUThreads, 1)
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kUOffBar);
   uint64_t *kv_full = bar, *kv_empty = bar + kUKS, *a_full = bar + 2 * kUKS,
            *a_empty = a_full + kUAS, *snap_full = a_empty + kUAS, *snap_done = snap_full + kUF,
-           *drain = snap_done + kUF;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(drain + 2);
+           *drain = snap_done + kUF, *d_ready = drain + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(d_ready + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(d_ready + 2);
+  static_assert((2 * kUKS + 2 * kUAS + 2 * kUF + 4) * 8 <= 256, "barrier region");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -139,6 +141,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
       mbar_init(&snap_done[f], 4);
     }
     mbar_init(drain, 1);
+    mbar_init(d_ready, 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -184,12 +187,16 @@ __global__ void __launch_bounds__(kUThreads, 1)
     // ---------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, kNP, false, false);
-      uint32_t it = 0, events = 0;
+      uint32_t it = 0, events = 0, items = 0;
       bool after_event = false;
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items) {
         const int batch = item % p.n_batches;
         const int nmt = min(kUF, p.n_mt - batch * kUF);
+        if (p.cont) {  // the epilogue has loaded the item's initial state into TMEM
+          if (!(ok = mbar_wait(d_ready, items & 1, abort_flag, p.err))) break;
+          tc_fence_after();
+        }
         for (int s = 0; ok && s < nsub; ++s, ++it) {
           const int ks = it % kUKS, as = it % kUAS;
           // a_full also covers kv_full: every generator warp waited on kv_full[ks]
@@ -216,7 +223,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
             for (int f = 0; f < kUF; ++f)
               if (f < nmt)
                 mma_bf16_ts(tmem + f * kNP, tmem + kUColA + (as * kUF + f) * (kUT / 2) + 8 * k, bd,
-                            idesc, (s > 0 || k > 0) ? 1u : 0u);
+                            idesc, (s > 0 || k > 0 || p.cont) ? 1u : 0u);
           }
           after_event = false;
           // one commit per step: the generators release the K^T / V^T stage
@@ -242,10 +249,38 @@ __global__ void __launch_bounds__(kUThreads, 1)
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
       const int hb = item / p.n_batches, batch = item % p.n_batches;
+      if (p.cont) {
+        // continued prefill: S' = S_0 / w into the TMEM tiles (the item's MMAs
+        // accumulate onto it), and the snapshot before chunk 0 (slot 0) is
+        // w^2 S' = w S_0.  This thread writes the same state rows at the end.
+        for (int f = 0; f < kUF; ++f) {
+          const int mt = batch * kUF + f;
+          if (mt >= p.n_mt) continue;
+          const int slot = mt * 128 + lane_slot(row);
+          const float w = p.slot_w[slot];
+          const int r = p.row_of_slot[slot];
+          const float *src = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * 65;
+          __nv_bfloat16 *sdst = p.snap + ((size_t)hb * p.nsnap * 65) * p.m_pad + slot;
+          uint32_t v[kNP];
+#pragma unroll
+          for (int n = 0; n < kNP; ++n) {
+            const float x = (n < 65 && r >= 0) ? src[n] : 0.f;
+            v[n] = __float_as_uint(w != 0.f ? x / w : 0.f);
+            if (n < 65) sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(w * x);
+          }
+#pragma unroll
+          for (int j = 0; j < kNP / 16; ++j)
+            tmem_st16(tmem + tl + f * kNP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(d_ready);
+      }
       for (int s = 0; ok && s < nsub; ++s) {
         if (!is_event(s)) continue;
         const bool boundary = s != nsub - 1;
-        const int c = boundary ? (s + 1) / sub_per_chunk - 1 : 0;
+        const int c = boundary ? (s + 1) / sub_per_chunk - 1 + p.cont : 0;
         for (int f = 0; ok && f < kUF; ++f) {
           if (!(ok = mbar_wait(&snap_full[f], events & 1, abort_flag, p.err))) break;
           tc_fence_after();
@@ -386,6 +421,7 @@ struct RParams {
   GenWeights W;
   int n_tiles;
   int N, C, nsnap, head0;
+  int cont;    // 1: snapshot slot 0 holds the state before chunk 0
   float *out;  // [BH][N][64]
   int *err;
 };
@@ -418,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int chunk = t0 / p.C;
   const int c0 = chunk * p.C;
   const int nkb = (t0 - c0) / kKB + 128 / kKB;  // key blocks from the chunk start through t0+127
-  const bool inter = chunk > 0;
+  const bool inter = chunk > 0 || p.cont != 0;
 
   if (inter)
     for (int i = threadIdx.x; i < p.n_tiles; i += kThreads) sTiles[i] = p.tiles[i];
@@ -463,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&b_full[st], nt * kRB);
         for (int t = 0; t < nt; ++t)
           tma_load_3d(sB + (st * kRTS + t) * kRB, &tmS, &b_full[st], 64 * (kRTS * i + t), 0,
-                      hrel * p.nsnap + chunk - 1);
+                      hrel * p.nsnap + chunk - 1 + p.cont);
       }
       for (int j = max(0, i - kRBS); j < i; ++j) {
         volatile int never = 0;
@@ -705,7 +741,7 @@ bool tc_supported(int dK, int dV, int P, bool bf16) {
 }
 
 int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, float *state,
-                      int B, int H, int N, const DeviceBasis *basis, int *err,
+                      int B, int H, int N, bool cont, const DeviceBasis *basis, int *err,
                       cudaStream_t stream) {
   const int BH = B * H;
   const int n_tiles = basis->n_tiles;  // even, padded
@@ -716,7 +752,9 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
   // in-chunk quadratic part behind its inter-chunk MMAs; 4096 measured fastest
   // of 1024 / 2048 / 4096 at 16384 tokens.
   const int C = N <= kChunk ? ((N + 127) / 128) * 128 : kChunk;
-  const int nsnap = (N + C - 1) / C - 1;
+  // snapshots: the state before each chunk but the first, plus (continued
+  // prefill) the initial state before chunk 0 in slot 0
+  const int nsnap = (N + C - 1) / C - 1 + (cont ? 1 : 0);
   const int Npad = ((N + kUT - 1) / kUT) * kUT;  // multiple of the 128-token step
   const size_t snap_head = (size_t)nsnap * 65 * m_pad * 2;
   const size_t kt_head = (size_t)65 * Npad * 2;  // K^T or V^T of one head
@@ -776,6 +814,7 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
     up.n_batches = n_batches;
     up.n_items = g * n_batches;
     up.head0 = h0;
+    up.cont = cont ? 1 : 0;
     up.snap = snap;
     up.state = state;
     up.err = err;
@@ -790,6 +829,7 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
     rp.C = C;
     rp.nsnap = nsnap;
     rp.head0 = h0;
+    rp.cont = cont ? 1 : 0;
     rp.out = out;
     rp.err = err;
     if (nsnap == 0) mS = mQ;  // never read: no chunk has a predecessor

@@ -252,9 +252,12 @@ extern "C" const char *sata_kernel_name(int id) {
   return "unknown";
 }
 
-extern "C" int sata_prefill(const void *q, const void *k, const void *v, float *out,
-                            float *state, int B, int H, int N, int dK, int dV, int P,
-                            sata_dtype dt, sata_stream_t stream) {
+namespace {
+
+// sata_prefill (cont = false) and sata_prefill_continue (cont = true).
+int prefill_impl(const void *q, const void *k, const void *v, float *out, float *state, int B,
+                 int H, int N, int dK, int dV, int P, sata_dtype dt, sata_stream_t stream,
+                 bool cont) {
   if (!q || !k || !v || !out || !state) return SATA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state))
     return SATA_ERR_INVALID_ARG;
@@ -280,10 +283,25 @@ extern "C" int sata_prefill(const void *q, const void *k, const void *v, float *
   if (!force_simt && tc_supported(dK, dV, P, bf16) && basis->tile_desc) {
     int *err = device_error_ptr();
     if (!err) return SATA_ERR_NOMEM;
-    return launch_prefill_tc(q, k, v, out, state, B, H, N, basis, err, (cudaStream_t)stream);
-  }
-  return launch_prefill_simt(q, k, v, out, state, B, H, N, dK, dV, P, bf16, basis,
+    return launch_prefill_tc(q, k, v, out, state, B, H, N, cont, basis, err,
                              (cudaStream_t)stream);
+  }
+  return launch_prefill_simt(q, k, v, out, state, B, H, N, dK, dV, P, bf16, cont, basis,
+                             (cudaStream_t)stream);
+}
+
+}  // namespace
+
+extern "C" int sata_prefill(const void *q, const void *k, const void *v, float *out,
+                            float *state, int B, int H, int N, int dK, int dV, int P,
+                            sata_dtype dt, sata_stream_t stream) {
+  return prefill_impl(q, k, v, out, state, B, H, N, dK, dV, P, dt, stream, false);
+}
+
+extern "C" int sata_prefill_continue(const void *q, const void *k, const void *v, float *out,
+                                     float *state, int B, int H, int N, int dK, int dV, int P,
+                                     sata_dtype dt, sata_stream_t stream) {
+  return prefill_impl(q, k, v, out, state, B, H, N, dK, dV, P, dt, stream, true);
 }
 
 extern "C" int sata_decode_step(const void *q, const void *k, const void *v, float *state,

@@ -54,14 +54,15 @@ int read_and_clear_device_error();
 int *device_error_ptr();
 
 // ------------------------------------------------------------ launchers
+// cont: start from the state in `state` (continued prefill) instead of zero.
 int launch_prefill_simt(const void *q, const void *k, const void *v, float *out,
                         float *state, int B, int H, int N, int dK, int dV, int P,
-                        bool bf16, const DeviceBasis *basis, cudaStream_t stream);
+                        bool bf16, bool cont, const DeviceBasis *basis, cudaStream_t stream);
 
 // Tensor-core prefill (bf16, dK = dV = 64, P = 4); basis must carry the tile order.
 bool tc_supported(int dK, int dV, int P, bool bf16);
 int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, float *state,
-                      int B, int H, int N, const DeviceBasis *basis, int *err,
+                      int B, int H, int N, bool cont, const DeviceBasis *basis, int *err,
                       cudaStream_t stream);
 
 int launch_decode(const void *q, const void *k, const void *v, float *state, float *out,

@@ -105,6 +105,16 @@ def test_invalid_calls_rejected_on_host():
     assert pre(st=4 * A + 16) == sata.SATA_ERR_INVALID_ARG        # state overlaps out
     assert pre(N=1 << 30, B=4) == sata.SATA_ERR_INVALID_ARG      # index range
 
+    def cont(q=A, k=2 * A, v=3 * A, out=4 * A, st=5 * A, **kw):
+        a = {**args, **kw}
+        return L.sata_prefill_continue(q, k, v, out, st, a["B"], a["H"], a["N"], a["dK"],
+                                       a["dV"], a["P"], a["dt"], None)
+
+    assert cont(st=None) == sata.SATA_ERR_INVALID_ARG
+    assert cont(v=3 * A + 8) == sata.SATA_ERR_INVALID_ARG        # misaligned
+    assert cont(P=5) == sata.SATA_ERR_UNSUPPORTED
+    assert cont(st=4 * A + 16) == sata.SATA_ERR_INVALID_ARG       # state overlaps out
+
     def dec(q=A, k=2 * A, v=3 * A, st=5 * A, out=4 * A, **kw):
         a = {**args, **kw}
         return L.sata_decode_step(q, k, v, st, out, a["B"], a["H"], a["dK"], a["dV"], a["P"],

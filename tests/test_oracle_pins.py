@@ -253,6 +253,23 @@ def test_decode_continues_prefill():
     np.testing.assert_allclose(S, S_ref, rtol=1e-12, atol=1e-12)
 
 
+def test_feature_form_continues_from_a_state():
+    # a continued prefill: the per-token procedure started from the state of
+    # the first N0 tokens gives, for the later tokens, the definition's rows
+    # over the whole sequence, and the whole sequence's state
+    N0, N1 = 20, 17
+    q, k, v = make_qkv(2, 3, N0 + N1, 8, 4, seed=21)
+    S0 = oracle.final_state(k[:, :, :N0], v[:, :, :N0], 4)
+    num, den, out, S = oracle.feature_form(q[:, :, N0:], k[:, :, N0:], v[:, :, N0:], 4, state0=S0)
+    num_f, den_f, out_f = oracle.quadratic_form(q, k, v, 4)
+    np.testing.assert_allclose(num, num_f[:, :, N0:], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(den, den_f[:, :, N0:], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(S, oracle.final_state(k, v, 4), rtol=1e-12, atol=1e-12)
+    # from a zero state it is the plain prefill
+    z = oracle.feature_form(q, k, v, 4, state0=np.zeros_like(S))
+    np.testing.assert_allclose(z[2], out_f, rtol=1e-10, atol=1e-12)
+
+
 def test_error_against_softmax_shrinks_with_P():
     # [SATA-eng] "精度与效率的权衡参数": a higher truncation order is more accurate.
     q, k, v = workload_inputs(2)

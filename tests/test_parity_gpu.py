@@ -142,6 +142,83 @@ def test_prefill_then_decode_equals_longer_prefill(dt):
                            state_full.cpu().double().numpy()) <= 10 * TOL["f32"]
 
 
+def check_continue(B, H, N0, N1, dK, dV, P, dt, seed):
+    """GPU prefill of N0 tokens, then a continued prefill of N1 more: the later
+    outputs against the definition over all N0 + N1 tokens, the state against
+    the whole sequence's state."""
+    q, k, v = make_qkv(B, H, N0 + N1, dK, dV, seed=seed, dtype=dt)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    _, state = sata.prefill(qc[:, :, :N0].contiguous(), kc[:, :, :N0].contiguous(),
+                            vc[:, :, :N0].contiguous(), P)
+    out = sata.prefill_continue(qc[:, :, N0:].contiguous(), kc[:, :, N0:].contiguous(),
+                                vc[:, :, N0:].contiguous(), state, P)
+    torch.cuda.synchronize()
+    num, den, ref = oracle.quadratic_form(q, k, v, P)
+    cond = oracle.conditioning(q, k, P)
+    err, excluded = out_row_error(out.cpu().double().numpy(), ref[:, :, N0:], den[:, :, N0:],
+                                  cond[:, :, N0:])
+    assert excluded <= max(4, B * H * N1 // 200), excluded
+    assert err <= TOL[dt], (err, TOL[dt])
+    S = state.cpu().double().numpy()
+    assert state_col_error(S, oracle.final_state(k, v, P)) <= TOL[dt]
+    assert np.all(S[..., 0, -1] == N0 + N1)
+
+
+@pytest.mark.parametrize("B,H,N0,N1,dK,dV,P,dt", [
+    (2, 2, 300, 500, 16, 8, 4, "f32"),     # CUDA-core path, several chunks after the prefix
+    (1, 3, 1, 1, 8, 8, 3, "f32"),          # one token each
+    (1, 1, 700, 90, 32, 32, 4, "bf16"),    # CUDA-core path, bf16 inputs
+])
+def test_prefill_continue(B, H, N0, N1, dK, dV, P, dt):
+    check_continue(B, H, N0, N1, dK, dV, P, dt, seed=N0 + 7 * N1)
+
+
+@pytest.mark.parametrize("N0,N1", [
+    (4224, 4300),   # prefix with one snapshot; continuation crosses a chunk boundary
+    (100, 50),      # short prefix, single-chunk continuation
+])
+def test_prefill_continue_tensor_core(N0, N1):
+    check_continue(1, 2, N0, N1, 64, 64, 4, "bf16", seed=N0 + N1)
+
+
+@pytest.mark.parametrize("dt,dK", [("bf16", 64), ("f32", 16)])
+def test_prefill_continue_from_zero_is_prefill(dt, dK):
+    q, k, v = make_qkv(1, 2, 1500, dK, dK, seed=5, dtype=dt)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    out0, state0 = sata.prefill(qc, kc, vc, 4)
+    state = torch.zeros_like(state0)
+    out1 = sata.prefill_continue(qc, kc, vc, state, 4)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(out1, out0, rtol=1e-5, atol=1e-6)
+    torch.testing.assert_close(state, state0, rtol=1e-5, atol=1e-6)
+
+
+def test_serving_loop_prefill_decode_continue():
+    # prompt -> two decode steps -> more prompt -> one decode step, against one
+    # pass of the definition over the whole sequence
+    N0, N1, P = 200, 150, 4
+    q, k, v = make_qkv(2, 2, N0 + 3 + N1, 16, 16, seed=77)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    outs = []
+    o, state = sata.prefill(qc[:, :, :N0].contiguous(), kc[:, :, :N0].contiguous(),
+                            vc[:, :, :N0].contiguous(), P)
+    outs.append(o)
+    for i in (N0, N0 + 1):
+        outs.append(sata.decode_step(qc[:, :, i].contiguous(), kc[:, :, i].contiguous(),
+                                     vc[:, :, i].contiguous(), state, P)[:, :, None])
+    a, b = N0 + 2, N0 + 2 + N1
+    outs.append(sata.prefill_continue(qc[:, :, a:b].contiguous(), kc[:, :, a:b].contiguous(),
+                                      vc[:, :, a:b].contiguous(), state, P))
+    outs.append(sata.decode_step(qc[:, :, b].contiguous(), kc[:, :, b].contiguous(),
+                                 vc[:, :, b].contiguous(), state, P)[:, :, None])
+    torch.cuda.synchronize()
+    got = torch.cat([x.cpu() for x in outs], dim=2).double().numpy()
+    num, den, ref = oracle.quadratic_form(q, k, v, P)
+    err, _ = out_row_error(got, ref, den, oracle.conditioning(q, k, P))
+    assert err <= TOL["f32"], err
+    assert state_col_error(state.cpu().double().numpy(), oracle.final_state(k, v, P)) <= TOL["f32"]
+
+
 def test_workload5_decode():
     """Workload 5: bf16 prefill N=8192 for B=32,H=8 (dK=dV=64, P=4), then 1024
     decode steps.  Oracle: two sampled heads over every step from the oracle's
