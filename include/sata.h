@@ -33,8 +33,9 @@
  *   - Arguments are validated on the host before anything is launched; an
  *     invalid call returns a status and launches nothing.  Nothing throws
  *     across this interface.
- *   - Supported: dK, dV in {8, 16, 32, 64}; 1 <= P <= 4; B, H, N >= 1 with
- *     B*H*N*max(dK,dV) < 2^31.
+ *   - Supported: dK, dV in {8, 16, 32, 64}; 1 <= P <= 5 (P = 5 adds the
+ *     degree-4 tensor: m = C(dK+4, 4), e.g. 814385 rows at dK = 64, and runs
+ *     on CUDA cores); B, H, N >= 1 with B*H*N*max(dK,dV) < 2^31.
  *   - The library lazily allocates, per device, its basis tables and a
  *     grow-only scratch workspace (cudaMalloc); both live until sata_release()
  *     or process exit.  Calls from several host threads are serialised by an
@@ -125,7 +126,8 @@ int sata_decode_step(const void *q, const void *k, const void *v, float *state,
  * memory: hosts whose caching allocator owns the whole GPU, serving loops
  * that must not hit cudaMalloc/cudaFree because those can synchronise the
  * device, plug-in hosts whose policy forbids library-side allocations.)
- * Same arguments, layouts, semantics and results as sata_decode_step.  It
+ * Same arguments, layouts, semantics and results as sata_decode_step, for
+ * P <= 4 (its static tables hold degrees 0..3; P = 5 -> SATA_ERR_UNSUPPORTED).  It
  * calls no cudaMalloc, cudaFree or other allocating routine: its scratch (the
  * per-head partial sums) is a file-scope __device__ array of
  * SATA_NOALLOC_MAX_PARTIALS floats (256 KiB), and its basis tables are static

@@ -69,7 +69,7 @@ HostBasis build_host_basis(int dK, int P) {
         }
       }
       b.degree.push_back((uint8_t)p);
-      for (int s = 0; s < 3; ++s) b.ix.push_back((uint8_t)(s < p ? t[s] : dK));
+      for (int s = 0; s < 4; ++s) b.ix.push_back((uint8_t)(s < p ? t[s] : dK));
       b.weight.push_back(1.0 / std::sqrt(fact * std::pow((double)dK, 0.5 * p)));
       ++b.m;
       more = (p > 0) && next_sorted_tuple(t, p, dK);

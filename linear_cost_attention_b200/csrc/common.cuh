@@ -21,11 +21,21 @@ __device__ __forceinline__ float taylor_trunc(float s, int P) {
   return t;
 }
 
+// Packed basis row (i1 | i2 << 7 | i3 << 14 | i4 << 21 | degree << 28).
+__device__ __forceinline__ int packed_index(uint32_t packed, int s) {
+  return (packed >> (7 * s)) & 0x7f;
+}
+__device__ __forceinline__ int packed_degree(uint32_t packed) { return packed >> 28; }
+// The packed row of a padding slot: every index at x[dK] (its weight is 0).
+__host__ __device__ constexpr uint32_t padding_row(int dK) {
+  return (uint32_t)dK | (uint32_t)dK << 7 | (uint32_t)dK << 14 | (uint32_t)dK << 21;
+}
+
 // phi_r(x) for one basis row from the packed table entry (unused index slots
 // point at x[dK] == 1.0f).
 __device__ __forceinline__ float feature_from_packed(const float *x, uint32_t packed, float w) {
-  const int i1 = packed & 0xff, i2 = (packed >> 8) & 0xff, i3 = (packed >> 16) & 0xff;
-  return w * x[i1] * x[i2] * x[i3];
+  return w * x[packed_index(packed, 0)] * x[packed_index(packed, 1)] *
+         x[packed_index(packed, 2)] * x[packed_index(packed, 3)];
 }
 
 }  // namespace sata

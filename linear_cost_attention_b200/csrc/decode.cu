@@ -62,10 +62,10 @@ __global__ void __launch_bounds__(D1 *DecodeShape<D1>::KB)
     const int bh = (int)(r / m);
     const int a = (int)(r - (long long)bh * m);
     const uint32_t pk = idx[a];
-    const int deg = pk >> 24;
+    const int deg = packed_degree(pk);
     float fq = w[a], fk = fq;
     for (int s = 0; s < deg; ++s) {
-      const int ii = (pk >> (8 * s)) & 0xff;
+      const int ii = packed_index(pk, s);
       fq *= to_f32(q[(size_t)bh * dK + ii]);
       fk *= to_f32(k[(size_t)bh * dK + ii]);
     }

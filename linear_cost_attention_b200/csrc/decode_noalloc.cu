@@ -68,8 +68,7 @@ int noalloc_setup(int dev, NoAllocDevice **out) {
     std::vector<uint32_t> idx(hb.m);
     std::vector<float> w(hb.m);
     for (int64_t r = 0; r < hb.m; ++r) {
-      idx[r] = (uint32_t)hb.ix[3 * r] | (uint32_t)hb.ix[3 * r + 1] << 8 |
-               (uint32_t)hb.ix[3 * r + 2] << 16 | (uint32_t)hb.degree[r] << 24;
+      idx[r] = pack_row(hb, r);
       w[r] = (float)hb.weight[r];
     }
     if (cudaMemcpy(d.idx + kTableOffset[s], idx.data(), hb.m * sizeof(uint32_t),

@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(kThreads)
   const size_t bh = (size_t)head0 + blockIdx.y;
   if (tid < kFT) {
     const int a = a0 + tid;
-    sidx[tid] = a < m ? idx[a] : (uint32_t)(DK | DK << 8 | DK << 16);
+    sidx[tid] = a < m ? idx[a] : padding_row(DK);
     sw[tid] = a < m ? w[a] : 0.f;
   }
   float acc[R];
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kThreads)
       __syncthreads();
       if (tid < kFT) {
         const int a = a0 + tid;
-        sidx[tid] = a < m ? idx[a] : (uint32_t)(DK | DK << 8 | DK << 16);
+        sidx[tid] = a < m ? idx[a] : padding_row(DK);
         sw[tid] = a < m ? w[a] : 0.f;
       }
       for (int e = tid; e < kFT * D1; e += kThreads) {

@@ -62,8 +62,7 @@ const DeviceBasis *get_device_basis(int dK, int P, int *status) {
   std::vector<uint32_t> idx(hb.m);
   std::vector<float> w(hb.m);
   for (int64_t r = 0; r < hb.m; ++r) {
-    idx[r] = (uint32_t)hb.ix[3 * r] | (uint32_t)hb.ix[3 * r + 1] << 8 |
-             (uint32_t)hb.ix[3 * r + 2] << 16 | (uint32_t)hb.degree[r] << 24;
+    idx[r] = pack_row(hb, r);
     w[r] = (float)hb.weight[r];
   }
   DeviceBasis *db = new DeviceBasis();
@@ -100,7 +99,7 @@ const DeviceBasis *get_device_basis(int dK, int P, int *status) {
       if (r < 0) continue;
       uint32_t v = 0;
       for (int q = 0; q < 3; ++q) {
-        const int ii = q < hb.degree[r] ? hb.ix[3 * r + q] : 64;
+        const int ii = q < hb.degree[r] ? hb.ix[4 * r + q] : 64;
         v |= (uint32_t)ii << (8 * q);
       }
       sidx[k] = v;
@@ -263,7 +262,7 @@ int prefill_impl(const void *q, const void *k, const void *v, float *out, float 
     return SATA_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1) return SATA_ERR_INVALID_ARG;
   if (dt != SATA_F32 && dt != SATA_BF16) return SATA_ERR_INVALID_ARG;
-  if (!supported_dim(dK) || !supported_dim(dV) || P < 1 || P > 4) return SATA_ERR_UNSUPPORTED;
+  if (!supported_dim(dK) || !supported_dim(dV) || P < 1 || P > kMaxP) return SATA_ERR_UNSUPPORTED;
   const long long BHN = (long long)B * H * N;
   if (BHN * (dK > dV ? dK : dV) >= (1LL << 31)) return SATA_ERR_INVALID_ARG;
   const int64_t m = count_basis(dK, P);
@@ -312,7 +311,7 @@ extern "C" int sata_decode_step(const void *q, const void *k, const void *v, flo
     return SATA_ERR_INVALID_ARG;
   if (B < 1 || H < 1) return SATA_ERR_INVALID_ARG;
   if (dt != SATA_F32 && dt != SATA_BF16) return SATA_ERR_INVALID_ARG;
-  if (!supported_dim(dK) || !supported_dim(dV) || P < 1 || P > 4) return SATA_ERR_UNSUPPORTED;
+  if (!supported_dim(dK) || !supported_dim(dV) || P < 1 || P > kMaxP) return SATA_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
   const int64_t m = count_basis(dK, P);
   if (BH * m * (dV + 1) >= (1LL << 40)) return SATA_ERR_INVALID_ARG;

@@ -19,14 +19,23 @@ struct HostBasis {
   int dK = 0, P = 0;
   int64_t m = 0;
   std::vector<uint8_t> degree;          // [m]
-  std::vector<uint8_t> ix;              // [m*3]; unused slots = dK (points at a 1.0)
+  std::vector<uint8_t> ix;              // [m*4]; unused slots = dK (points at a 1.0)
   std::vector<double> weight;           // [m]  1/sqrt(alpha! * dK^(p/2))
 };
 HostBasis build_host_basis(int dK, int P);
 int64_t count_basis(int dK, int P);  // m, or -1
+constexpr int kMaxP = 5;             // degrees 0..4 (four index slots)
+
+// Packed row for the CUDA-core kernels: four 7-bit indices (unused slots = dK,
+// which points at a 1.0) and the degree in bits 28..30.
+inline uint32_t pack_row(const HostBasis &hb, int64_t r) {
+  uint32_t v = (uint32_t)hb.degree[r] << 28;
+  for (int s = 0; s < 4; ++s) v |= (uint32_t)hb.ix[4 * r + s] << (7 * s);
+  return v;
+}
 
 // Device copy of the tables in the packed form the kernels read.
-//   idx[r] = i1 | i2 << 8 | i3 << 16 | degree << 24  (unused slots = dK)
+//   idx[r] = i1 | i2 << 7 | i3 << 14 | i4 << 21 | degree << 28  (unused slots = dK)
 //   w[r]   = fp32 weight
 struct DeviceBasis {
   int dK = 0, P = 0;

@@ -37,7 +37,7 @@ bool build_tile_order(int dK, TileOrder *out) {
   for (int64_t r = 0; r < hb.m; ++r) {
     const int deg = hb.degree[r];
     int ix[3] = {-1, -1, -1};
-    for (int s = 0; s < deg; ++s) ix[s] = hb.ix[3 * r + s];
+    for (int s = 0; s < deg; ++s) ix[s] = hb.ix[4 * r + s];
     lex[tuple_key(deg, ix[0], ix[1], ix[2])] = (int32_t)r;
   }
   std::vector<TileDesc> tiles;

@@ -66,7 +66,7 @@ int main() {
         double ref = 0.0;
         if (row_id >= 0) {
           ref = hb.weight[row_id];
-          for (int s = 0; s < hb.degree[row_id]; ++s) ref *= x[hb.ix[3 * row_id + s]];
+          for (int s = 0; s < hb.degree[row_id]; ++s) ref *= x[hb.ix[4 * row_id + s]];
         }
         const double err = std::fabs(got - ref);
         const double tol = 3 * std::ldexp(1.0, -8) * std::fabs(ref) + 1e-30;

@@ -99,7 +99,7 @@ def test_invalid_calls_rejected_on_host():
     assert pre(dt=7) == sata.SATA_ERR_INVALID_ARG
     assert pre(dK=12) == sata.SATA_ERR_UNSUPPORTED
     assert pre(dV=128) == sata.SATA_ERR_UNSUPPORTED
-    assert pre(P=5) == sata.SATA_ERR_UNSUPPORTED
+    assert pre(P=6) == sata.SATA_ERR_UNSUPPORTED
     assert pre(P=0) == sata.SATA_ERR_UNSUPPORTED
     assert pre(out=A) == sata.SATA_ERR_INVALID_ARG               # out aliases q
     assert pre(st=4 * A + 16) == sata.SATA_ERR_INVALID_ARG        # state overlaps out
@@ -112,7 +112,7 @@ def test_invalid_calls_rejected_on_host():
 
     assert cont(st=None) == sata.SATA_ERR_INVALID_ARG
     assert cont(v=3 * A + 8) == sata.SATA_ERR_INVALID_ARG        # misaligned
-    assert cont(P=5) == sata.SATA_ERR_UNSUPPORTED
+    assert cont(P=6) == sata.SATA_ERR_UNSUPPORTED
     assert cont(st=4 * A + 16) == sata.SATA_ERR_INVALID_ARG       # state overlaps out
 
     def dec(q=A, k=2 * A, v=3 * A, st=5 * A, out=4 * A, **kw):

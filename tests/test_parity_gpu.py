@@ -87,6 +87,9 @@ def test_workload4_bf16_sampled_heads():
     (3, 1, 129, 32, 32, 1, "f32"),      # P = 1: running mean
     (1, 2, 300, 64, 64, 2, "bf16"),
     (2, 2, 1100, 32, 32, 4, "bf16"),
+    (2, 2, 150, 8, 16, 5, "f32"),       # P = 5: degree-4 features (495 rows)
+    (1, 2, 700, 16, 16, 5, "bf16"),     # P = 5, several chunks (4845 rows)
+    (1, 1, 40, 64, 64, 5, "bf16"),      # P = 5 at dK = 64: 814385 rows, CUDA cores
 ])
 def test_edge_shapes(B, H, N, dK, dV, P, dt):
     q, k, v = make_qkv(B, H, N, dK, dV, seed=B * 1000 + N, dtype=dt)
@@ -111,14 +114,14 @@ def test_tensor_core_prefill_shapes(B, H, N):
 def test_invalid_call_raises():
     q = torch.zeros(1, 1, 4, 8, device="cuda")
     with pytest.raises(sata.SataError):
-        sata.prefill(q, q, q, P=5)
+        sata.prefill(q, q, q, P=6)
     with pytest.raises(sata.SataError):
         sata.sata_prefill(q, q, q, q, q, 1, 1, 4, 8, 8, 4, torch.float32)  # aliasing
 
 
-@pytest.mark.parametrize("dt", ["f32", "bf16"])
-def test_prefill_then_decode_equals_longer_prefill(dt):
-    B, H, N0, t, dK, dV, P = 2, 2, 96, 6, 16, 16, 4
+@pytest.mark.parametrize("dt,P", [("f32", 4), ("bf16", 4), ("f32", 5)])
+def test_prefill_then_decode_equals_longer_prefill(dt, P):
+    B, H, N0, t, dK, dV = 2, 2, 96, 6, 16, 16
     q, k, v = make_qkv(B, H, N0 + t, dK, dV, seed=31, dtype=dt)
     qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
     out_full, state_full = sata.prefill(qc, kc, vc, P)
