@@ -3,29 +3,36 @@
 // Same chunked decomposition as the CUDA-core path (prefill_simt.cu), with
 // both state contractions on the 5th-generation tensor cores:
 //
-//   tc_chunk_states  one CTA per (head, 4 x 128 basis rows): the four state
-//     tiles S[128 x 80] (dV+1 = 65 columns padded to the MMA's N = 80) stay in
-//     TMEM for the whole sequence.  Per 64 tokens: TMA brings K and V; eight
-//     generator warps write phi(K)^T (basis rows x tokens, MN-major) into
-//     shared memory, one thread per token; one thread issues
-//     S += phi(K)^T [V, 1] (M = 128, N = 80, K = 16 per instruction).  At every
-//     chunk boundary the epilogue warps copy S to a bf16 snapshot (the state
-//     before the next chunk, "恒定计算成本的工程实现": the fixed-size state), and
-//     after the last token write the fp32 state in lexicographic row order.
-//   tc_readout       one CTA per (head, 128 tokens of chunk c):
-//     D[128 x 80] = sum over 750 tiles of 64 basis rows of phi(Q_tile) S_(c-1)
-//     (phi(Q) generated per tile into shared memory, snapshot tiles streamed by
-//     TMA), plus the in-chunk part sum_{c0 <= j <= i} T_4(s_ij) [v_j, 1] per
+//   tc_transpose_kv  K, V [BH, N, 64] -> K^T, [V, 1]^T [BH, 65, Npad]: every
+//     basis monomial is a product of three K^T rows (row 64 = ones supplies the
+//     lower degrees) and [V, 1]^T is the K-major B operand of the state MMAs.
+//   tc_chunk_states  persistent CTAs (448 threads) over items = (head, two
+//     128-row state tiles); the tiles S'[128 x 80] (dV+1 = 65 columns padded
+//     to the MMA's N = 80) stay in TMEM for the whole sequence.  Per 128-token
+//     step: warp 0 brings the K^T and [V,1]^T boxes by TMA; warps 6-13 (one
+//     thread per basis row = TMEM lane) multiply three K^T rows for every
+//     token and store the unweighted monomials into a TMEM A stage; warp 1
+//     (one thread) issues 16 MMAs M = 128, N = 80, K = 16 (A from TMEM, B from
+//     shared memory), the two tiles alternating.  At each chunk boundary warps
+//     2-5 copy w^2 S' into a bf16 snapshot (the state before the next chunk,
+//     "恒定计算成本的工程实现": the fixed-size state); after the last token they
+//     write w S' as the fp32 state in lexicographic row order.  A continued
+//     prefill first loads S_0 / w into the tiles and S_0 w as snapshot 0.
+//   tc_readout       one CTA (512 threads) per (head, 128 tokens of chunk c):
+//     D[128 x 80] in TMEM accumulates phi(Q) S_(c-1) over 750 tiles of 64
+//     basis rows (warps 8-15, one thread per token = TMEM lane, generate the
+//     tiles' monomials into TMEM A stages; warp 0 streams the snapshot tiles by
+//     TMA) plus the in-chunk part sum_{c0 <= j <= i} T_4(s_ij) [v_j, 1] per
 //     64-key block: scores Q K^T into TMEM, T_4 and the causal mask by the
-//     epilogue warps, P split into bf16 hi + lo parts (T_4 rounded to bf16 loses
-//     too much on rows whose denominator cancels), P_hi [V, 1] + P_lo [V, 1]
-//     into D; out = D[:, :64] / D[:, 64].
+//     epilogue warps 4-7, P split into bf16 hi + lo parts (T_4 rounded to bf16
+//     loses too much on rows whose denominator cancels), P_hi [V, 1] +
+//     P_lo [V, 1] into D; out = D[:, :64] / D[:, 64].  Warp 2 brings Q and the
+//     chunk's K, V blocks by TMA.
 //
-// Warp roles (512 threads): 0 TMA producer, 1 MMA issuer (one thread) and TMEM
-// owner, 2 second TMA producer (readout), 4-7 epilogue (TMEM lane quarters),
-// 8-15 feature generators.  Every mbarrier wait is bounded (tc_common.cuh);
-// on a timeout the kernel records an error, drains what it issued and frees
-// its TMEM before returning.
+// The MMA-issuing thread waits on one barrier per stage: a wait there stalls
+// the tensor pipe, whose queue holds only a couple of MMAs.  Every mbarrier
+// wait is bounded (tc_common.cuh); on a timeout the kernel records an error,
+// drains what it issued and frees its TMEM before returning.
 #include <cuda.h>
 
 #include <algorithm>
