@@ -42,7 +42,7 @@ struct DeviceBasis {
   int64_t m = 0;
   uint32_t *idx = nullptr;
   float *w = nullptr;
-  // Tensor-core tile order (dK in {32, 64}, P == 4); null when not built.
+  // Tensor-core tile order (dK = 64, P == 4); null when not built.
   int n_tiles = 0;              // 64-feature tiles
   int64_t m_pad = 0;            // n_tiles * 64
   void *tile_desc = nullptr;      // [n_tiles] TileDesc (tile_order.h)
