@@ -28,6 +28,14 @@ constexpr int kFT = 32;  // basis rows per tile
 constexpr int kTT = 32;  // tokens per step
 constexpr int kTB = 32;  // query tokens per readout block
 
+// Register tile of a thread: 4 consecutive rows (basis rows, or tokens in the
+// readout) starting at 4 * (tid / 32) by the columns tid % 32 + 32 j < D1.
+// Per reduction step it reads its 4 row values with one broadcast 16-byte
+// shared load and one value per column, for 4 FMAs per column.
+constexpr int kRowsT = 4;
+static_assert(kThreads / 32 * kRowsT == kFT && kFT == kTT && kTT == kTB, "tile geometry");
+template <int D1> struct ColTile { static constexpr int n = (D1 + 31) / 32; };
+
 template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(kThreads)
     simt_chunk_states(const T *__restrict__ k, const T *__restrict__ v,
@@ -35,15 +43,15 @@ __global__ void __launch_bounds__(kThreads)
                       int m, int N, int C, int head0, float *__restrict__ snap, int nsnap,
                       int cont, float *__restrict__ state) {
   constexpr int D1 = DV + 1;
-  constexpr int ENT = kFT * D1;
-  constexpr int R = (ENT + kThreads - 1) / kThreads;
+  constexpr int RC = ColTile<D1>::n;
   __shared__ float ks[kTT][DK + 1];
   __shared__ float vs[kTT][D1];
-  __shared__ float ph[kTT][kFT + 1];
+  __shared__ __align__(16) float ph[kTT][kFT];  // ph[t][a]: row a of token t
   __shared__ uint32_t sidx[kFT];
   __shared__ float sw[kFT];
 
   const int tid = threadIdx.x;
+  const int ty = tid >> 5, tx = tid & 31;
   const int a0 = blockIdx.x * kFT;
   const size_t bh = (size_t)head0 + blockIdx.y;
   if (tid < kFT) {
@@ -51,16 +59,18 @@ __global__ void __launch_bounds__(kThreads)
     sidx[tid] = a < m ? idx[a] : padding_row(DK);
     sw[tid] = a < m ? w[a] : 0.f;
   }
-  float acc[R];
+  float acc[kRowsT][RC];
   float *st = state + bh * (size_t)m * D1;
+  // entry (row a0 + 4 ty + i, column tx + 32 j) of the tile, if it exists
+  auto live = [&](int i, int j) { return a0 + kRowsT * ty + i < m && tx + 32 * j < D1; };
+  auto at = [&](int i, int j) { return (size_t)(a0 + kRowsT * ty + i) * D1 + tx + 32 * j; };
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    // a continued prefill starts from the caller's state (read here, by the
-    // thread that overwrites the same entries at the end)
-    const int e = tid + r * kThreads;
-    acc[r] = 0.f;
-    if (cont && e < ENT && a0 + e / D1 < m) acc[r] = st[(size_t)(a0 + e / D1) * D1 + e % D1];
-  }
+  for (int i = 0; i < kRowsT; ++i)
+#pragma unroll
+    for (int j = 0; j < RC; ++j)
+      // a continued prefill starts from the caller's state (read here, by the
+      // thread that overwrites the same entries at the end)
+      acc[i][j] = (cont && live(i, j)) ? st[at(i, j)] : 0.f;
   const T *kh = k + bh * N * DK;
   const T *vh = v + bh * N * DV;
 
@@ -68,13 +78,10 @@ __global__ void __launch_bounds__(kThreads)
     if ((t0 > 0 || cont) && t0 % C == 0) {
       float *sp = snap + ((size_t)blockIdx.y * nsnap + (t0 / C - 1 + cont)) * (size_t)m * D1;
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int e = tid + r * kThreads;
-        if (e < ENT) {
-          const int a = e / D1, c = e % D1;
-          if (a0 + a < m) sp[(size_t)(a0 + a) * D1 + c] = acc[r];
-        }
-      }
+      for (int i = 0; i < kRowsT; ++i)
+#pragma unroll
+        for (int j = 0; j < RC; ++j)
+          if (live(i, j)) sp[at(i, j)] = acc[i][j];
     }
     __syncthreads();
     for (int e = tid; e < kTT * (DK + 1); e += kThreads) {
@@ -95,26 +102,23 @@ __global__ void __launch_bounds__(kThreads)
       ph[t][a] = feature_from_packed(ks[t], sidx[a], sw[a]);
     }
     __syncthreads();
+#pragma unroll 4
+    for (int t = 0; t < kTT; ++t) {
+      const float4 f = *reinterpret_cast<const float4 *>(&ph[t][kRowsT * ty]);
+      const float fr[kRowsT] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int e = tid + r * kThreads;
-      if (e < ENT) {
-        const int a = e / D1, c = e % D1;
-        float s = acc[r];
-#pragma unroll 8
-        for (int t = 0; t < kTT; ++t) s = fmaf(ph[t][a], vs[t][c], s);
-        acc[r] = s;
+      for (int j = 0; j < RC; ++j) {
+        const float x = (tx + 32 * j < D1) ? vs[t][tx + 32 * j] : 0.f;
+#pragma unroll
+        for (int i = 0; i < kRowsT; ++i) acc[i][j] = fmaf(fr[i], x, acc[i][j]);
       }
     }
   }
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int e = tid + r * kThreads;
-    if (e < ENT) {
-      const int a = e / D1, c = e % D1;
-      if (a0 + a < m) st[(size_t)(a0 + a) * D1 + c] = acc[r];
-    }
-  }
+  for (int i = 0; i < kRowsT; ++i)
+#pragma unroll
+    for (int j = 0; j < RC; ++j)
+      if (live(i, j)) st[at(i, j)] = acc[i][j];
 }
 
 template <int DK, int DV, typename T>
@@ -123,19 +127,20 @@ __global__ void __launch_bounds__(kThreads)
                  const uint32_t *__restrict__ idx, const float *__restrict__ w, int m, int N,
                  int C, int P, int head0, const float *__restrict__ snap, int nsnap,
                  int cont, float *__restrict__ out) {
-  static_assert(kTB == kFT && kTB == kTT, "tile sizes share shared-memory buffers");
   constexpr int D1 = DV + 1;
-  constexpr int ENT = kTB * D1;
-  constexpr int R = (ENT + kThreads - 1) / kThreads;
+  constexpr int RC = ColTile<D1>::n;
   __shared__ float qs[kTB][DK + 1];
   __shared__ float ks[kTT][DK + 1];
   __shared__ float vs[kTT][D1];
-  __shared__ float ph[kTB][kFT + 1];
+  // pt[r][t]: the reduction index r (basis row, or key) outer and the token
+  // contiguous, so a thread's 4 tokens are one 16-byte load
+  __shared__ __align__(16) float pt[kFT][kTB];
   __shared__ float sn[kFT][D1];
   __shared__ uint32_t sidx[kFT];
   __shared__ float sw[kFT];
 
   const int tid = threadIdx.x;
+  const int ty = tid >> 5, tx = tid & 31;
   const int t0 = blockIdx.x * kTB;
   const size_t bh = (size_t)head0 + blockIdx.y;
   const int chunk = t0 / C;
@@ -150,9 +155,25 @@ __global__ void __launch_bounds__(kThreads)
     if (i < DK) x = (t0 + t < N) ? to_f32(qh[(size_t)(t0 + t) * DK + i]) : 0.f;
     qs[t][i] = x;
   }
-  float acc[R];
+  float acc[kRowsT][RC];
 #pragma unroll
-  for (int r = 0; r < R; ++r) acc[r] = 0.f;
+  for (int i = 0; i < kRowsT; ++i)
+#pragma unroll
+    for (int j = 0; j < RC; ++j) acc[i][j] = 0.f;
+  // acc[i][j] += sum_r pt[r][4 ty + i] * b[r][tx + 32 j] over kFT reduction rows
+  auto accumulate = [&](const float (*b)[D1]) {
+#pragma unroll 4
+    for (int r = 0; r < kFT; ++r) {
+      const float4 f = *reinterpret_cast<const float4 *>(&pt[r][kRowsT * ty]);
+      const float fr[kRowsT] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int j = 0; j < RC; ++j) {
+        const float x = (tx + 32 * j < D1) ? b[r][tx + 32 * j] : 0.f;
+#pragma unroll
+        for (int i = 0; i < kRowsT; ++i) acc[i][j] = fmaf(fr[i], x, acc[i][j]);
+      }
+    }
+  };
 
   // inter-chunk: phi(q_i)^T S_(before chunk)
   if (chunk > 0 || cont) {
@@ -170,21 +191,11 @@ __global__ void __launch_bounds__(kThreads)
       }
       __syncthreads();
       for (int e = tid; e < kTB * kFT; e += kThreads) {
-        const int t = e / kFT, a = e % kFT;
-        ph[t][a] = feature_from_packed(qs[t], sidx[a], sw[a]);
+        const int t = e % kTB, a = e / kTB;
+        pt[a][t] = feature_from_packed(qs[t], sidx[a], sw[a]);
       }
       __syncthreads();
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int e = tid + r * kThreads;
-        if (e < ENT) {
-          const int t = e / D1, c = e % D1;
-          float s = acc[r];
-#pragma unroll 8
-          for (int a = 0; a < kFT; ++a) s = fmaf(ph[t][a], sn[a][c], s);
-          acc[r] = s;
-        }
-      }
+      accumulate(sn);
     }
   }
 
@@ -207,34 +218,24 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
     for (int e = tid; e < kTB * kTT; e += kThreads) {
-      const int t = e / kTT, j = e % kTT;
+      const int t = e % kTB, j = e / kTB;
       float s = 0.f;
 #pragma unroll
       for (int i = 0; i < DK; ++i) s = fmaf(qs[t][i], ks[j][i], s);
       const bool keep = (j0 + j <= t0 + t) && (j0 + j < jend);
-      ph[t][j] = keep ? taylor_trunc(s * scale, P) : 0.f;
+      pt[j][t] = keep ? taylor_trunc(s * scale, P) : 0.f;
     }
     __syncthreads();
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int e = tid + r * kThreads;
-      if (e < ENT) {
-        const int t = e / D1, c = e % D1;
-        float s = acc[r];
-#pragma unroll 8
-        for (int j = 0; j < kTT; ++j) s = fmaf(ph[t][j], vs[j][c], s);
-        acc[r] = s;
-      }
-    }
+    accumulate(vs);
   }
 
   // normalise
   __syncthreads();
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int e = tid + r * kThreads;
-    if (e < ENT) sn[e / D1][e % D1] = acc[r];
-  }
+  for (int i = 0; i < kRowsT; ++i)
+#pragma unroll
+    for (int j = 0; j < RC; ++j)
+      if (tx + 32 * j < D1) sn[kRowsT * ty + i][tx + 32 * j] = acc[i][j];
   __syncthreads();
   for (int e = tid; e < kTB * DV; e += kThreads) {
     const int t = e / DV, c = e % DV;
