@@ -270,6 +270,31 @@ def test_feature_form_continues_from_a_state():
     np.testing.assert_allclose(z[2], out_f, rtol=1e-10, atol=1e-12)
 
 
+def test_softmax_reference_matches_library_attention():
+    # the exact-softmax reference used by the error-vs-P pin is PyTorch's own
+    # causal scaled dot-product attention (same 1/sqrt(dK) scale), in fp64
+    import torch
+    q, k, v = make_qkv(2, 3, 70, 16, 8, seed=13)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double(), k.double(), v.double(), is_causal=True).numpy()
+    np.testing.assert_allclose(oracle.softmax_attention(q, k, v, row_block=32), ref,
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_conditioning_is_the_sum_of_absolute_kernel_values():
+    # brute force over (i, j <= i) with the scalar Taylor sum
+    q, k, _ = make_qkv(1, 2, 23, 4, 4, seed=17)
+    qd, kd = q.double().numpy(), k.double().numpy()
+    got = oracle.conditioning(q, k, 4, row_block=5)
+    for h in range(2):
+        for i in range(23):
+            want = 0.0
+            for j in range(i + 1):
+                s = float(qd[0, h, i] @ kd[0, h, j]) / 2.0
+                want += abs(1 + s + s * s / 2 + s ** 3 / 6)
+            assert abs(got[0, h, i] - want) <= 1e-12 * want
+
+
 def test_error_against_softmax_shrinks_with_P():
     # [SATA-eng] "精度与效率的权衡参数": a higher truncation order is more accurate.
     q, k, v = workload_inputs(2)
