@@ -127,6 +127,21 @@ def test_invalid_calls_rejected_on_host():
     assert dec(out=2 * A) == sata.SATA_ERR_INVALID_ARG
 
 
+def test_plain_c_program_uses_the_abi(tmp_path):
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    sata.lib()  # builds or finds the in-tree library
+    libdir = os.path.dirname(sata.LIB_PATH)
+    exe = tmp_path / "abi_c_check"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "cpu", "abi_c_check.c"), "-o", str(exe),
+                    "-L", libdir, "-lsata", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
 
