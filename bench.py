@@ -146,35 +146,32 @@ def source_sha(files=None) -> str:
 
 
 # --------------------------------------------------------------- oracle timing
-def oracle_prefill_sample(rows: int, seed: int = 0):
-    """fp64 oracle on a bounded sample of the prefill workload: `rows` query rows
-    (evenly spaced over N) of one head through the quadratic form, and the state
-    accumulation over `rows` tokens.  Returns (seconds, equivalent tokens)."""
-    import numpy as np
-
+def oracle_prefill_sample(n: int, seed: int = 0):
+    """The fp64 oracle on a bounded sample of the prefill workload: its
+    quadratic form (``oracle.quadratic_form``) over the first ``n`` tokens of
+    one head, then the final state (``oracle.final_state``) of those tokens.
+    Returns (seconds, tokens of the whole workload the same work is worth):
+    the quadratic form's cost grows with the number of (query, key) pairs, so
+    n tokens of one head are worth n(n+1)/2 of the H*N(N+1)/2 pairs; the
+    state's cost grows with the tokens (n of H*N)."""
     import oracle
     from sata_inputs import make_qkv
 
     w = PREFILL
-    q, k, v = make_qkv(1, 1, w["N"], w["dK"], w["dV"], seed=seed, dtype="bf16")
-    qq, kk, vv = (t.double().numpy()[0, 0] for t in (q, k, v))
-    idx = np.linspace(0, w["N"] - 1, rows).astype(np.int64)
+    q, k, v = make_qkv(1, 1, n, w["dK"], w["dV"], seed=seed, dtype="bf16")
     t0 = time.perf_counter()
-    scale = 1.0 / math.sqrt(w["dK"])
-    for i0 in range(0, rows, 256):
-        ii = idx[i0:i0 + 256]
-        s = (qq[ii] @ kk.T) * scale
-        t = oracle.taylor_kernel(s, w["P"])
-        t = np.where(np.arange(w["N"])[None, :] <= ii[:, None], t, 0.0)
-        _ = t @ vv, t.sum(axis=1)
-    oracle.final_state(k[:, :, :rows], v[:, :, :rows], w["P"])
-    dt = time.perf_counter() - t0
-    # one head of H: `rows` token rows count as rows/H tokens of the whole batch
-    return dt, rows / w["H"]
+    oracle.quadratic_form(q, k, v, w["P"])
+    t1 = time.perf_counter()
+    oracle.final_state(k, v, w["P"])
+    t2 = time.perf_counter()
+    full_pairs = w["H"] * w["N"] * (w["N"] + 1) / 2
+    full_tokens = w["B"] * w["H"] * w["N"]
+    t_full = (t1 - t0) * full_pairs / (n * (n + 1) / 2) + (t2 - t1) * full_tokens / n
+    return t2 - t0, w["B"] * w["N"] * (t2 - t0) / t_full
 
 
 def oracle_decode_sample(heads: int, seed: int = 1):
-    """fp64 oracle decode step on `heads` heads from a random state.  Returns
+    """``oracle.decode_step`` on `heads` heads from a random state.  Returns
     (seconds, equivalent tokens of the B=32,H=8 step)."""
     import numpy as np
 
@@ -193,29 +190,41 @@ def oracle_decode_sample(heads: int, seed: int = 1):
     return dt, heads / w["H"]
 
 
-def host_threads() -> int:
+def host_threads() -> dict:
+    """Host cores available to this process, and the threads numpy's BLAS
+    pool uses (the oracle's matrix products run there)."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count() or 1
+    blas = 1
     try:
         from threadpoolctl import threadpool_info
 
         info = threadpool_info()
-        return max(int(i.get("num_threads", 1)) for i in info) if info else 1
+        blas = max(int(i.get("num_threads", 1)) for i in info) if info else 1
     except Exception:
-        return 1
+        pass
+    return {"cores": cores, "numpy_threads": blas}
 
 
 def cpu_baseline(budget_s: float = 20.0):
-    rows = 2048
-    dt, tok = oracle_prefill_sample(rows)
-    while dt < budget_s * 0.4 and rows < PREFILL["N"]:
-        rows = min(PREFILL["N"], rows * 2)
-        dt, tok = oracle_prefill_sample(rows)
+    oracle_prefill_sample(256)  # first-call set-up (thread pools, tables) untimed
+    n = 2048
+    dt, tok = oracle_prefill_sample(n)
+    while dt < budget_s * 0.25 and n < PREFILL["N"]:
+        n = min(PREFILL["N"], n * 2)
+        dt, tok = oracle_prefill_sample(n)
     ddt, dtok = oracle_decode_sample(2)
-    return {"value": tok / dt, "unit": "tokens/s", "cores": host_threads(), "kind": "oracle",
-            "sample": f"prefill: {rows} query rows evenly spaced over N=16384 of 1 of 8 heads "
-                      f"(quadratic form) + state over {rows} tokens, fp64 numpy, {dt:.1f} s",
+    th = host_threads()
+    return {"value": tok / dt, "unit": "tokens/s", "cores": th["cores"],
+            "numpy_threads": th["numpy_threads"], "kind": "oracle",
+            "sample": f"prefill: oracle.quadratic_form + oracle.final_state on the first {n} "
+                      f"tokens of 1 of the 8 heads (fp64 numpy, {dt:.1f} s), scaled to the "
+                      f"workload by (query, key) pairs and by tokens respectively",
             "decode": {"value": dtok / ddt, "unit": "tokens/s",
-                       "sample": f"1 decode step of 2 of the 256 heads from a random state, "
-                                 f"{ddt:.2f} s"}}
+                       "sample": f"oracle.decode_step on 2 of the 256 heads from a random "
+                                 f"state, {ddt:.2f} s"}}
 
 
 # --------------------------------------------------------------- ranks
@@ -454,17 +463,19 @@ def run_ours(args, rank, world, local_rank):
 # --------------------------------------------------------------- reference arm
 def run_reference(args):
     per_step = []
-    rows = args.ref_rows
+    n = args.ref_tokens
     for i in range(args.warmup + args.steps):
-        dt, tok = oracle_prefill_sample(rows, seed=i)
+        dt, tok = oracle_prefill_sample(n, seed=i)
         if i >= args.warmup:
             per_step.append((dt, tok))
     t = sum(d for d, _ in per_step)
     tok = sum(x for _, x in per_step)
     ddt, dtok = oracle_decode_sample(2)
     value = tok / t
-    sample = (f"each step: {rows} query rows evenly spaced over N=16384 of 1 of 8 heads "
-              f"(quadratic form) + state over {rows} tokens; fp64 numpy on host cores")
+    th = host_threads()
+    sample = (f"each step: oracle.quadratic_form + oracle.final_state on the first {n} tokens "
+              f"of 1 of 8 heads, fp64 numpy on the host cores, scaled to the workload by "
+              f"(query, key) pairs and by tokens")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -473,10 +484,11 @@ def run_reference(args):
         "data": "synthetic: seeded i.i.d. N(0,1) q,k,v cast to bf16",
         "config": {"workload": WORKLOAD, "global_batch": PREFILL["B"] * PREFILL["H"],
                    "seq_len": PREFILL["N"], "parallelism": "host threads"},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_threads(),
-                         "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": th["cores"],
+                         "numpy_threads": th["numpy_threads"], "kind": "oracle",
+                         "sample": sample},
         "decode": {"value": dtok / ddt, "unit": "tokens/s",
-                   "sample": "1 decode step of 2 of 256 heads from a random state"},
+                   "sample": "oracle.decode_step on 2 of 256 heads from a random state"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -504,6 +516,13 @@ def profile_case(case: str):
         qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
         for _ in range(3):
             sata.prefill(qd, kd, vd, P)
+    elif case == "prefill_full":
+        # the benchmark's prefill workload itself (about 0.4 GB on the device)
+        w = PREFILL
+        q, k, v = make_qkv(w["B"], w["H"], w["N"], w["dK"], w["dV"], seed=4, dtype="bf16")
+        qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+        for _ in range(3):
+            sata.prefill(qd, kd, vd, w["P"])
     else:
         raise SystemExit(f"unknown profile case {case}")
     torch.cuda.synchronize()
@@ -517,9 +536,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=128)
-    ap.add_argument("--ref-rows", type=int, default=1024)
+    ap.add_argument("--ref-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["decode", "prefill"], default=None,
+    ap.add_argument("--profile-case", choices=["decode", "prefill", "prefill_full"], default=None,
                     help="run a small case of one kernel for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:

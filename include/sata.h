@@ -38,8 +38,15 @@
  *     on CUDA cores); B, H, N >= 1 with B*H*N*max(dK,dV) < 2^31.
  *   - The library lazily allocates, per device, its basis tables and a
  *     grow-only scratch workspace (cudaMalloc); both live until sata_release()
- *     or process exit.  Calls from several host threads are serialised by an
- *     internal mutex.
+ *     or process exit.  The first call on a device for a given (dK, P) builds
+ *     the tables and waits for the device (cudaDeviceSynchronize): make it
+ *     before any stream capture.
+ *   - Thread safety: every prefill and decode call holds one internal
+ *     (recursive) mutex from validation through its last launch, and the
+ *     caches and the profiling records are read and written only under it,
+ *     so calls from several host threads are serialised on the host (the
+ *     work they enqueue runs in stream order on the GPU).
+ *     sata_decode_step_noalloc is the exception; see its notes.
  */
 #ifndef SATA_H_
 #define SATA_H_
@@ -138,9 +145,11 @@ int sata_decode_step(const void *q, const void *k, const void *v, float *state,
  *   - B*H*(dV+1) > SATA_NOALLOC_MAX_PARTIALS (e.g. more than 1008 heads at
  *     dV = 64) -> SATA_ERR_INVALID_ARG, nothing launched.
  *   - The first call on a device does a one-time set-up with that device
- *     current (resolves the arrays' device addresses with
- *     cudaGetSymbolAddress and copies the basis tables in, synchronously);
- *     make that first call before any stream capture.
+ *     current: it resolves the arrays' device addresses with
+ *     cudaGetSymbolAddress, copies the basis tables in and waits for the
+ *     device (cudaDeviceSynchronize), so the tables are complete for a first
+ *     call on any stream; make that first call before any stream capture.
+ *   - Unlike the other calls it does not take the library's call lock.
  *   - All calls on a device share the scratch, which keeps the last call's
  *     contents; each call clears what it uses first.  Calls that overlap on
  *     the GPU (other streams or host threads) race on it: order them. */
@@ -149,6 +158,17 @@ int sata_decode_step_noalloc(const void *q, const void *k, const void *v,
                              float *state, float *out, int B, int H, int dK,
                              int dV, int P, sata_dtype dt,
                              sata_stream_t stream);
+
+/* Test hook (no counterpart on the pages).  Bounds every wait of a role in
+ * the tensor-core prefill kernels (a producer, the MMA issuer, an epilogue or
+ * generator warp waiting for another role) to `cycles` SM clock cycles;
+ * cycles <= 0 restores the default bound (about 2 s).  A wait that runs out
+ * records SATA_ERR_TIMEOUT for sata_get_error, makes every role of its CTA
+ * leave its loop, and the CTA still waits (with the default bound) for its
+ * own copies and MMAs in flight and frees its TMEM before it exits; the
+ * call's outputs are then incomplete.  Used by the tests to exercise that
+ * path.  Returns the previous setting.  Host only. */
+long long sata_test_set_wait_limit(long long cycles);
 
 /* Synchronises `stream`, then reports (and clears) the first device-side error
  * recorded by this library's kernels on the current device (a bounded wait

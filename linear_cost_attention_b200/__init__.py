@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
     L.sata_profile_read.restype = i
     L.sata_kernel_name.argtypes = [i]
     L.sata_kernel_name.restype = ctypes.c_char_p
+    L.sata_test_set_wait_limit.argtypes = [ctypes.c_longlong]
+    L.sata_test_set_wait_limit.restype = ctypes.c_longlong
     _lib = L
     return L
 
@@ -181,6 +183,12 @@ def sata_profile_read(cap: int = 64):
 
 def sata_kernel_name(kid: int) -> str:
     return lib().sata_kernel_name(int(kid)).decode()
+
+
+def sata_test_set_wait_limit(cycles: int) -> int:
+    """Test hook: bound the tensor-core kernels' role waits to ``cycles``
+    (<= 0 restores the default).  Returns the previous setting."""
+    return int(lib().sata_test_set_wait_limit(int(cycles)))
 
 
 # ------------------------------------------------------------- conveniences

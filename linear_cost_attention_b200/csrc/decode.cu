@@ -157,10 +157,10 @@ __global__ void __launch_bounds__(D1 *DecodeShape<D1>::KB)
 template <int D1>
 __global__ void decode_finalize(const float *__restrict__ y, float *__restrict__ out, int BH) {
   constexpr int DV = D1 - 1;
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= BH * DV) return;
-  const int bh = i / DV, c = i % DV;
-  out[i] = y[(size_t)bh * D1 + c] / y[(size_t)bh * D1 + DV];
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)BH * DV) return;
+  const long long bh = i / DV, c = i % DV;
+  out[i] = y[bh * D1 + c] / y[bh * D1 + DV];
 }
 
 template <int D1, typename T>

@@ -47,7 +47,9 @@ int dim_slot(int d) { return d == 8 ? 0 : d == 16 ? 1 : d == 32 ? 2 : d == 64 ? 
 
 // Once per device, with that device current: resolve the arrays' device
 // addresses (in host code the array names are host-side stand-ins, not device
-// addresses) and fill the tables.  Synchronous.
+// addresses) and fill the tables.  Synchronous: it returns after the copies
+// have landed (cudaDeviceSynchronize), so a first call made on any stream sees
+// complete tables.
 int noalloc_setup(int dev, NoAllocDevice **out) {
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   NoAllocDevice &d = g_noalloc_dev[dev];
@@ -78,6 +80,14 @@ int noalloc_setup(int dev, NoAllocDevice **out) {
       cudaGetLastError();
       return SATA_ERR_CUDA;
     }
+  }
+  // cudaMemcpy from pageable host memory can return once the data is staged,
+  // before the DMA lands, and kernels on a non-blocking stream (any
+  // torch.cuda.Stream) are not ordered after the legacy stream: wait for the
+  // copies before the tables can be read by any launch.
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return SATA_ERR_CUDA;
   }
   d.ready = true;
   *out = &d;

@@ -88,6 +88,7 @@ constexpr int kUGenWarps = 4 * kUF;
 constexpr int kUEpiWarp0 = 2, kUGenWarp0 = 6;  // warps 2..5 epilogue, 6.. generators
 constexpr int kUThreads = 32 * (kUGenWarp0 + kUGenWarps);
 constexpr int kMaxTiles = 768;  // tile table capacity in smem (readout)
+constexpr int kMaxDevices = 64;  // per-device launch attributes
 constexpr int kChunk = 4096;    // tokens per chunk (a multiple of the 128-token step)
 constexpr uint32_t kUColA = 160;               // TMEM: D at f*80, A from column 160
 constexpr uint32_t kUTmemCols = 512;
@@ -117,6 +118,7 @@ struct UParams {
   __nv_bfloat16 *snap;  // [G][nsnap][65][m_pad]; slot 0 = initial state if cont
   float *state;         // [BH][m][65]
   int *err;
+  long long wait_limit;  // cycles before a role's wait gives up (drains: full limit)
 };
 
 __global__ void __launch_bounds__(kUThreads, 1)
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
         for (int s = 0; s < nsub; ++s, ++it) {
           const int st = it % kUKS;
           if (it >= kUKS &&
-              !(ok = mbar_wait(&kv_empty[st], ((it / kUKS) - 1) & 1, abort_flag, p.err)))
+              !(ok = mbar_wait(&kv_empty[st], ((it / kUKS) - 1) & 1, abort_flag, p.err, p.wait_limit)))
             break;
           mbar_arrive_expect_tx(&kv_full[st], 2 * 65 * kRow + 2 * kUVTh);
           for (int h = 0; h < 2; ++h) {
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
         const int batch = item % p.n_batches;
         const int nmt = min(kUF, p.n_mt - batch * kUF);
         if (p.cont) {  // the epilogue has loaded the item's initial state into TMEM
-          if (!(ok = mbar_wait(d_ready, items & 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(d_ready, items & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
         }
         for (int s = 0; ok && s < nsub; ++s, ++it) {
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
           // a_full also covers kv_full: every generator warp waited on kv_full[ks]
           // before arriving.  One barrier wait per step: a wait in this thread
           // stalls until the MMAs already issued have drained.
-          if (!(ok = mbar_wait(&a_full[as], (it / kUAS) & 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&a_full[as], (it / kUAS) & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
           const uint32_t b0 = smem_u32(sVT + ks * kUVT);
           const bool event = is_event(s);
@@ -217,7 +219,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
             // every tile's barrier is waited once per event, in order, so no
             // barrier can run two phases ahead of its waiter
             for (int f = 0; ok && f < kUF; ++f)
-              ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err);
+              ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err, p.wait_limit);
             if (!ok) break;
             tc_fence_after();
           }
@@ -289,7 +291,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
         const bool boundary = s != nsub - 1;
         const int c = boundary ? (s + 1) / sub_per_chunk - 1 + p.cont : 0;
         for (int f = 0; ok && f < kUF; ++f) {
-          if (!(ok = mbar_wait(&snap_full[f], events & 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&snap_full[f], events & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
           const int mt = batch * kUF + f;
           const bool live = mt < p.n_mt;
@@ -341,9 +343,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
       const uint32_t si = (ix & 7), sj = ((ix >> 8) & 7), sl = ((ix >> 16) & 7);
       for (int s = 0; ok && s < nsub; ++s, ++it) {
         const int ks = it % kUKS, as = it % kUAS;
-        if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err))) break;
+        if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err, p.wait_limit))) break;
         if (it >= kUAS) {
-          if (!(ok = mbar_wait(&a_empty[as], ((it / kUAS) - 1) & 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&a_empty[as], ((it / kUAS) - 1) & 1, abort_flag, p.err, p.wait_limit))) break;
           // the MMAs of step it - kUAS are complete and this warp read its K^T
           // rows long ago: release that step's K^T / V^T stage
           __syncwarp();
@@ -431,6 +433,7 @@ struct RParams {
   int cont;    // 1: snapshot slot 0 holds the state before chunk 0
   float *out;  // [BH][N][64]
   int *err;
+  long long wait_limit;  // cycles before a role's wait gives up (drains: full limit)
 };
 
 __device__ __forceinline__ float taylor4(float s) {
@@ -500,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int i = 0;
       for (; i < n_stages; ++i) {
         const int st = i % kRBS;
-        if (i >= kRBS && !mbar_wait(&b_empty[st], ((i / kRBS) - 1) & 1, abort_flag, p.err))
+        if (i >= kRBS && !mbar_wait(&b_empty[st], ((i / kRBS) - 1) & 1, abort_flag, p.err, p.wait_limit))
           break;
         const int nt = min(kRTS, p.n_tiles - kRTS * i);
         mbar_arrive_expect_tx(&b_full[st], nt * kRB);
@@ -523,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(sQ, &tmQ, q_full, 0, t0, bh);
       int kb = 0;
       for (; kb < nkb; ++kb) {
-        if (kb > 0 && !mbar_wait(kv_empty, (kb - 1) & 1, abort_flag, p.err)) break;
+        if (kb > 0 && !mbar_wait(kv_empty, (kb - 1) & 1, abort_flag, p.err, p.wait_limit)) break;
         mbar_arrive_expect_tx(kv_full, 2 * kRKV);
         tma_load_3d(sK, &tmK, kv_full, 0, c0 + kKB * kb, bh);
         tma_load_3d(sV, &tmV, kv_full, 0, c0 + kKB * kb, bh);
@@ -542,13 +545,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int kb_qk = 0, kb_pv = 0;
       const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV);
       const uint32_t p0 = smem_u32(sP), lbo_v = smem_u32(sOnes) - v0;
-      ok = mbar_wait(q_full, 0, abort_flag, p.err);
+      ok = mbar_wait(q_full, 0, abort_flag, p.err, p.wait_limit);
       // in-chunk part, advanced whenever its inputs are ready
       auto intra = [&](bool block) {
         while (ok && kb_pv < nkb) {
           if (kb_qk == kb_pv) {  // next: scores of block kb_qk
             if (block) {
-              if (!(ok = mbar_wait(kv_full, kb_qk & 1, abort_flag, p.err))) return;
+              if (!(ok = mbar_wait(kv_full, kb_qk & 1, abort_flag, p.err, p.wait_limit))) return;
             } else if (!mbar_test_wait(kv_full, kb_qk & 1)) {
               return;
             }
@@ -561,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++kb_qk;
           } else {  // next: P [V, 1] of block kb_pv
             if (block) {
-              if (!(ok = mbar_wait(p_full, kb_pv & 1, abort_flag, p.err))) return;
+              if (!(ok = mbar_wait(p_full, kb_pv & 1, abort_flag, p.err, p.wait_limit))) return;
             } else if (!mbar_test_wait(p_full, kb_pv & 1)) {
               return;
             }
@@ -587,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = i % kRStages, bs = i % kRBS;
           // a_full also covers b_full: the generator warps wait on the snapshot
           // stage before arriving (one barrier wait per stage in this thread)
-          if (!(ok = mbar_wait(&a_full[st], (i / kRStages) & 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&a_full[st], (i / kRStages) & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
           const int nt = min(kRTS, p.n_tiles - kRTS * i);
           for (int t = 0; t < nt; ++t) {
@@ -604,11 +607,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (ok) intra(true);
-      mma_commit(o_full);  // also orders every MMA before the final TMEM release
-      if (!ok) {
-        volatile int never = 0;
-        mbar_wait(o_full, 0, &never, p.err);
-      }
+      // o_full tracks every MMA of this thread: wait for it here whatever
+      // happened, so that no MMA is in flight when the CTA frees its TMEM (the
+      // epilogue's own wait on it may have given up)
+      mma_commit(o_full);
+      volatile int never = 0;
+      mbar_wait(o_full, 0, &never, p.err);
     }
   } else if (warp >= 4 && warp < 8) {
     // ---------------- epilogue: in-chunk Taylor scores, then normalisation
@@ -618,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
     bool ok = true;
     for (int kb = 0; ok && kb < nkb; ++kb) {
-      if (!(ok = mbar_wait(s_full, kb & 1, abort_flag, p.err))) break;
+      if (!(ok = mbar_wait(s_full, kb & 1, abort_flag, p.err, p.wait_limit))) break;
       tc_fence_after();
       {
         uint32_t v[kKB];
@@ -647,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok && (ok = mbar_wait(o_full, 0, abort_flag, p.err))) {
+    if (ok && (ok = mbar_wait(o_full, 0, abort_flag, p.err, p.wait_limit))) {
       tc_fence_after();
       uint32_t v[kNP];
 #pragma unroll
@@ -670,13 +674,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gw = warp - 8;
     const int half = gw >> 2;
     const int row = lane + 32 * (gw & 3);
-    bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
+    bool ok = mbar_wait(q_full, 0, abort_flag, p.err, p.wait_limit);
     const uint8_t *qrow = sQ + row * kRow;
     const int n_stages = (p.n_tiles + kRTS - 1) / kRTS;
     for (int i = 0; ok && i < n_stages; ++i) {
       const int st = i % kRStages;
       if (i >= kRStages && !(ok = mbar_wait(&a_empty[st], ((i / kRStages) - 1) & 1, abort_flag,
-                                            p.err)))
+                                            p.err, p.wait_limit)))
         break;
 #pragma unroll 1
       for (int t = half; t < kRTS; t += 2) {
@@ -694,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st32(tmem + ((uint32_t)(32 * (gw & 3)) << 16) + kRColA + (st * kRTS + t) * 32, out);
       }
       tmem_st_wait();
-      if (!(ok = mbar_wait(&b_full[i % kRBS], (i / kRBS) & 1, abort_flag, p.err))) break;
+      if (!(ok = mbar_wait(&b_full[i % kRBS], (i / kRBS) & 1, abort_flag, p.err, p.wait_limit))) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&a_full[st]);
@@ -779,17 +783,21 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
   if (!make_map(&mV64, v, 64, N, BH, 64) || !make_map(&mK64, k, 64, N, BH, 64) ||
       !make_map(&mQ, q, 64, N, BH, 128))
     return SATA_ERR_CUDA;
-  static bool attr_done = false;
-  if (!attr_done) {
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  // The >48 KiB dynamic shared-memory opt-in is a per-device attribute: set it
+  // once for every device this process prefills on.  (Callers hold the
+  // library's call lock, so the flags need no lock of their own.)
+  static bool attr_done[kMaxDevices] = {};
+  if (dev < 0 || dev >= kMaxDevices) return SATA_ERR_CUDA;
+  if (!attr_done[dev]) {
     if (cudaFuncSetAttribute(tc_chunk_states, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kUSmem) != cudaSuccess ||
         cudaFuncSetAttribute(tc_readout, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmem) !=
             cudaSuccess)
       return SATA_ERR_CUDA;
-    attr_done = true;
+    attr_done[dev] = true;
   }
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
 
   const int n_mt = m_pad / 128;
@@ -825,6 +833,7 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
     up.snap = snap;
     up.state = state;
     up.err = err;
+    up.wait_limit = tc_wait_limit();
     prof_kernel_begin(stream, K_TC_CHUNK_STATES);
     tc_chunk_states<<<std::min(up.n_items, nsm), kUThreads, kUSmem, stream>>>(mKT, mVT, up);
     prof_kernel_end(stream);
@@ -839,6 +848,7 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
     rp.cont = cont ? 1 : 0;
     rp.out = out;
     rp.err = err;
+    rp.wait_limit = tc_wait_limit();
     if (nsnap == 0) mS = mQ;  // never read: no chunk has a predecessor
     prof_kernel_begin(stream, K_TC_READOUT);
     tc_readout<<<dim3((N + 127) / 128, g), kThreads, kRSmem, stream>>>(mQ, mK64, mV64, mS, rp);

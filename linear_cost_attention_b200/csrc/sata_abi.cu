@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "sata_internal.h"
+#include "tc_common.cuh"
 #include "tile_order.h"
 
 namespace sata {
@@ -21,7 +22,9 @@ struct DeviceCache {
   int *err = nullptr;  // device error word
 };
 
-std::mutex g_mutex;
+// Guards the caches and the profiling records, and is held for the whole of
+// every prefill / decode call (recursive: the call's helpers lock it again).
+std::recursive_mutex g_mutex;
 std::map<int, DeviceCache> g_devices;
 
 DeviceCache &cache_for_current_device(int *dev_out) {
@@ -54,7 +57,7 @@ void free_basis(DeviceBasis *b) {
 }  // namespace
 
 const DeviceBasis *get_device_basis(int dK, int P, int *status) {
-  std::lock_guard<std::mutex> lock(g_mutex);
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
   DeviceCache &dc = cache_for_current_device(nullptr);
   auto it = dc.bases.find({dK, P});
   if (it != dc.bases.end()) return it->second;
@@ -118,7 +121,12 @@ const DeviceBasis *get_device_basis(int dK, int P, int *status) {
          cudaMemcpy(db->tile_row, to.row_of_slot.data(), to.row_of_slot.size() * sizeof(int32_t),
                     cudaMemcpyHostToDevice) == cudaSuccess;
   }
+  // cudaMemcpy from pageable memory may return before the DMA has landed, and
+  // kernels on a non-blocking stream are not ordered after the legacy stream:
+  // finish the copies before any launch can read the tables.
+  if (ok && cudaDeviceSynchronize() != cudaSuccess) ok = false;
   if (!ok) {
+    cudaGetLastError();
     free_basis(db);
     *status = SATA_ERR_NOMEM;
     return nullptr;
@@ -128,7 +136,7 @@ const DeviceBasis *get_device_basis(int dK, int P, int *status) {
 }
 
 void *get_workspace(cudaStream_t stream, size_t bytes, int *status) {
-  std::lock_guard<std::mutex> lock(g_mutex);
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
   DeviceCache &dc = cache_for_current_device(nullptr);
   auto &ws = dc.workspaces[stream];
   if (ws.second >= bytes && ws.first) return ws.first;
@@ -152,7 +160,7 @@ void *get_workspace(cudaStream_t stream, size_t bytes, int *status) {
 }
 
 int *device_error_ptr() {
-  std::lock_guard<std::mutex> lock(g_mutex);
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
   DeviceCache &dc = cache_for_current_device(nullptr);
   if (!dc.err) {
     if (cudaMalloc(&dc.err, sizeof(int)) != cudaSuccess) {
@@ -160,7 +168,14 @@ int *device_error_ptr() {
       dc.err = nullptr;
       return nullptr;
     }
-    cudaMemset(dc.err, 0, sizeof(int));
+    // zeroed before any kernel (on any stream) can record into it
+    if (cudaMemset(dc.err, 0, sizeof(int)) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(dc.err);
+      dc.err = nullptr;
+      return nullptr;
+    }
   }
   return dc.err;
 }
@@ -170,7 +185,8 @@ int read_and_clear_device_error() {
   if (!p) return 0;
   int h = 0;
   if (cudaMemcpy(&h, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return -1;
-  if (h) cudaMemset(p, 0, sizeof(int));
+  if (h && (cudaMemset(p, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess))
+    return -1;
   return h;
 }
 
@@ -196,12 +212,14 @@ cudaEvent_t prof_event() {
 }  // namespace
 
 void prof_call_begin() {
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
   if (!g_prof_on) return;
   g_prof.clear();
   g_next_event = 0;
 }
 
 void prof_kernel_begin(cudaStream_t s, int id) {
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
   if (!g_prof_on) return;
   ProfRec r{id, prof_event(), prof_event()};
   if (r.a) cudaEventRecord(r.a, s);
@@ -209,6 +227,7 @@ void prof_kernel_begin(cudaStream_t s, int id) {
 }
 
 void prof_kernel_end(cudaStream_t s) {
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
   if (!g_prof_on || g_prof.empty()) return;
   if (g_prof.back().b) cudaEventRecord(g_prof.back().b, s);
 }
@@ -218,14 +237,14 @@ void prof_kernel_end(cudaStream_t s) {
 using namespace sata;
 
 extern "C" int sata_profile_enable(int on) {
-  std::lock_guard<std::mutex> lock(g_mutex);
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
   const int prev = g_prof_on ? 1 : 0;
   g_prof_on = on != 0;
   return prev;
 }
 
 extern "C" int sata_profile_read(float *ms_out, int *ids_out, int cap) {
-  std::lock_guard<std::mutex> lock(g_mutex);
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
   const int n = (int)g_prof.size();
   for (int i = 0; i < n && i < cap; ++i) {
     float ms = 0.f;
@@ -273,6 +292,7 @@ int prefill_impl(const void *q, const void *k, const void *v, float *out, float 
       overlaps(state, ns, q, nq) || overlaps(state, ns, k, nq) || overlaps(state, ns, v, nv) ||
       overlaps(out, no, state, ns))
     return SATA_ERR_INVALID_ARG;
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);  // one call at a time
   int st = SATA_OK;
   const DeviceBasis *basis = get_device_basis(dK, P, &st);
   if (!basis) return st;
@@ -315,6 +335,8 @@ extern "C" int sata_decode_step(const void *q, const void *k, const void *v, flo
   const long long BH = (long long)B * H;
   const int64_t m = count_basis(dK, P);
   if (BH * m * (dV + 1) >= (1LL << 40)) return SATA_ERR_INVALID_ARG;
+  // head and output indices are 32-bit in the kernels
+  if (BH * (dK > dV + 1 ? dK : dV + 1) >= (1LL << 31)) return SATA_ERR_INVALID_ARG;
   const size_t es = dt == SATA_F32 ? 4 : 2;
   const size_t nq = BH * dK * es, nv = BH * dV * es, no = BH * dV * 4;
   const size_t ns = (size_t)BH * m * (dV + 1) * 4;
@@ -322,6 +344,7 @@ extern "C" int sata_decode_step(const void *q, const void *k, const void *v, flo
       overlaps(state, ns, q, nq) || overlaps(state, ns, k, nq) || overlaps(state, ns, v, nv) ||
       overlaps(out, no, state, ns))
     return SATA_ERR_INVALID_ARG;
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);  // one call at a time
   int st = SATA_OK;
   const DeviceBasis *basis = get_device_basis(dK, P, &st);
   if (!basis) return st;
@@ -341,6 +364,23 @@ extern "C" int sata_get_error(sata_stream_t stream) {
   return code == 0 ? SATA_OK : SATA_ERR_TIMEOUT;
 }
 
+namespace sata {
+namespace {
+long long g_tc_wait_limit = 0;  // 0: the kernels' full limit
+}  // namespace
+long long tc_wait_limit() {
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
+  return g_tc_wait_limit > 0 ? g_tc_wait_limit : tc::kWaitLimitCycles;
+}
+}  // namespace sata
+
+extern "C" long long sata_test_set_wait_limit(long long cycles) {
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
+  const long long prev = g_tc_wait_limit;
+  g_tc_wait_limit = cycles > 0 ? cycles : 0;
+  return prev;
+}
+
 extern "C" const char *sata_status_string(int status) {
   switch (status) {
     case SATA_OK: return "SATA_OK";
@@ -354,7 +394,7 @@ extern "C" const char *sata_status_string(int status) {
 }
 
 extern "C" void sata_release(void) {
-  std::lock_guard<std::mutex> lock(g_mutex);
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
   int cur = 0;
   cudaGetDevice(&cur);
   for (auto &kv : g_devices) {

@@ -70,6 +70,9 @@ int launch_prefill_simt(const void *q, const void *k, const void *v, float *out,
 
 // Tensor-core prefill (bf16, dK = dV = 64, P = 4); basis must carry the tile order.
 bool tc_supported(int dK, int dV, int P, bool bf16);
+// Cycles a role's wait in the tensor-core kernels may take before it gives up
+// (default: the kernels' full limit; lowered only by sata_test_set_wait_limit).
+long long tc_wait_limit();
 int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, float *state,
                       int B, int H, int N, bool cont, const DeviceBasis *basis, int *err,
                       cudaStream_t stream);

@@ -83,18 +83,19 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up when
-// *abort becomes non-zero or after kWaitLimitCycles; on a timeout it records
+// *abort becomes non-zero or after `limit` cycles; on a timeout it records
 // kErrWaitTimeout in *err and sets *abort so every role leaves its loop.
-// Returns false when the caller must stop.
+// Returns false when the caller must stop.  The waits that drain a CTA's own
+// copies and MMAs before it exits always use the full kWaitLimitCycles.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int *err) {
+                                          int *err, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 0) {
       if (*abort) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > limit) {
         atomicCAS(err, 0, kErrWaitTimeout);
         *abort = 1;
         return false;

@@ -21,7 +21,7 @@ Sources (web pages; cited by title and section):
   (mokono.cn), section "2.1 标准注意力实现与瓶颈分析": layout
   (batch, heads, seq_len, dim) and score scale dim**-0.5.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 degrees 0..P-1; inclusive causal mask j <= i; one normaliser shared by all
 degrees; no eps, clamp or max-subtraction; weights 1/sqrt(alpha! d_K^(p/2))
 (square root of the multinomial count times the Taylor 1/p! and the score

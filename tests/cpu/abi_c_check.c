@@ -26,6 +26,9 @@ int main(void) {
       SATA_ERR_INVALID_ARG)
     return 9;
   if (sata_status_string(SATA_ERR_UNSUPPORTED) == NULL) return 10;
+  /* the test hook keeps and returns its setting (host only) */
+  if (sata_test_set_wait_limit(1000) != 0) return 11;
+  if (sata_test_set_wait_limit(0) != 1000) return 12;
   printf("ok\n");
   return 0;
 }

@@ -125,6 +125,8 @@ def test_invalid_calls_rejected_on_host():
     assert dec(H=0) == sata.SATA_ERR_INVALID_ARG
     assert dec(dK=7) == sata.SATA_ERR_UNSUPPORTED
     assert dec(out=2 * A) == sata.SATA_ERR_INVALID_ARG
+    # head and output indices are 32-bit in the kernels: B*H*(dV+1) < 2^31
+    assert dec(B=1 << 25, P=1, dV=64) == sata.SATA_ERR_INVALID_ARG
 
 
 def test_plain_c_program_uses_the_abi(tmp_path):

@@ -15,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import linear_cost_attention_b200 as sata
 from sata_inputs import make_qkv
 from tests.parity import TOL, state_col_error
@@ -39,6 +40,8 @@ def _row_err(a, b):
 @pytest.mark.parametrize("dt,B,H,dK,dV,P", [
     ("f32", 2, 4, 64, 64, 4),
     ("bf16", 3, 2, 32, 16, 3),
+    ("f32", 2, 2, 8, 8, 4),      # the dK = 8 table slot
+    ("bf16", 1, 3, 16, 32, 4),   # the dK = 16 table slot
 ])
 def test_noalloc_matches_regular_entry_point_two_calls(dt, B, H, dK, dV, P):
     N0 = 40
@@ -51,6 +54,7 @@ def test_noalloc_matches_regular_entry_point_two_calls(dt, B, H, dK, dV, P):
     out_na = torch.empty(B, H, dV, device="cuda")
     steps = [tuple(t[:, :, N0 + s].contiguous() for t in (qd, kd, vd)) for s in range(2)]
     torch.cuda.synchronize()
+    S_before = state.double().cpu().numpy()
     free_after_first = None
     for s, (qt, kt, vt) in enumerate(steps):
         sata.sata_decode_step(qt, kt, vt, s_ref, out_ref, B, H, dK, dV, P, q.dtype)
@@ -59,6 +63,13 @@ def test_noalloc_matches_regular_entry_point_two_calls(dt, B, H, dK, dV, P):
         assert _row_err(out_na, out_ref) <= TOL[dt], s
         assert state_col_error(s_na.double().cpu().numpy(),
                                s_ref.double().cpu().numpy()) <= TOL[dt], s
+        # and against the oracle's decode step from the state before this call
+        ref, S_or = oracle.decode_step(qt.cpu(), kt.cpu(), vt.cpu(), S_before, P)
+        got = out_na.double().cpu().numpy()
+        assert float(np.max(np.max(np.abs(got - ref), axis=-1) /
+                            np.max(np.abs(ref), axis=-1))) <= TOL[dt], s
+        assert state_col_error(s_na.double().cpu().numpy(), S_or) <= TOL[dt], s
+        S_before = s_na.double().cpu().numpy()
         if s == 0:
             free_after_first = torch.cuda.mem_get_info()[0]
     # the second call allocated nothing (allocation granularity is 2 MiB)
@@ -76,3 +87,70 @@ def test_noalloc_rejects_sizes_beyond_the_static_scratch():
     st = L.sata_decode_step_noalloc(None, 2 * A, 3 * A, 1 << 40, 4 * A, 1008, 1, 64, 64, 4, 1,
                                     None)
     assert st == sata.SATA_ERR_INVALID_ARG
+
+
+def test_noalloc_alone_on_a_side_stream_allocates_nothing():
+    """Only the allocation-free entry point, on a non-default stream: after one
+    warm-up call (module loading), repeated calls leave free device memory
+    exactly unchanged, and the result matches the oracle."""
+    B, H, dK, dV, P, N0 = 4, 2, 32, 32, 4, 30
+    q, k, v = make_qkv(B, H, N0 + 4, dK, dV, seed=303, dtype="bf16")
+    S0 = oracle.final_state(k[:, :, :N0], v[:, :, :N0], P)  # the state of a 30-token prefix
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        state = torch.from_numpy(S0).float().cuda()
+        out = torch.empty(B, H, dV, device="cuda")
+        toks = [tuple(t[:, :, N0 + i].contiguous().cuda() for t in (q, k, v)) for i in range(4)]
+    side.synchronize()
+    S_or = S0
+    sata.sata_decode_step_noalloc(*toks[0], state, out, B, H, dK, dV, P, q.dtype, side)
+    _, S_or = oracle.decode_step(q[:, :, N0], k[:, :, N0], v[:, :, N0], S_or, P)
+    side.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for i in range(1, 4):
+        sata.sata_decode_step_noalloc(*toks[i], state, out, B, H, dK, dV, P, q.dtype, side)
+        ref, S_or = oracle.decode_step(q[:, :, N0 + i], k[:, :, N0 + i], v[:, :, N0 + i], S_or,
+                                       P)
+        side.synchronize()
+        assert _row_err(out, torch.from_numpy(ref)) <= TOL["bf16"], i
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert state_col_error(state.double().cpu().numpy(), S_or) <= TOL["bf16"]
+
+
+_FRESH = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import oracle, linear_cost_attention_b200 as sata
+from sata_inputs import make_qkv
+torch.cuda.set_device(0)
+B, H, dK, dV, P, N0 = 2, 3, 16, 16, 4, 50
+q, k, v = make_qkv(B, H, N0 + 1, dK, dV, seed=808, dtype="f32")
+S0 = torch.from_numpy(oracle.final_state(k[:, :, :N0], v[:, :, :N0], P)).float()  # 50-token prefix
+side = torch.cuda.Stream()
+with torch.cuda.stream(side):
+    st = S0.cuda(); out = torch.empty(B, H, dV, device="cuda")
+    qt, kt, vt = (t[:, :, N0].contiguous().cuda() for t in (q, k, v))
+side.synchronize()
+# the library's first call in this process: its one-time set-up runs here
+sata.sata_decode_step_noalloc(qt, kt, vt, st, out, B, H, dK, dV, P, q.dtype, side)
+side.synchronize()
+ref, _ = oracle.decode_step(q[:, :, N0], k[:, :, N0], v[:, :, N0], S0, P)
+got = out.double().cpu().numpy()
+e = np.max(np.max(np.abs(got - ref), axis=-1) / np.max(np.abs(ref), axis=-1))
+print("err", e)
+sys.exit(0 if e <= 1e-4 else 1)
+"""
+
+
+def test_noalloc_first_call_of_a_fresh_process_on_a_side_stream():
+    """The one-time set-up (symbol addresses, table copies) must be complete
+    before the first kernel reads the tables, even when that kernel runs on a
+    non-blocking stream that is not ordered after the legacy stream."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _FRESH, root], capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, (r.stdout, r.stderr)
