@@ -365,82 +365,105 @@ def run_ours(args, rank, world, local_rank):
            "d2h_bytes_per_step": out.numel() * 4 + state.numel() * 4}
     del qd, kd, vd, out, state, q, k, v, qh, kh, vh, out_h, st_h
 
-    # ---------------- decode
+    # ---------------- decode: fp32 state and mixed-precision state
     dw = DECODE
     dm = basis_m(dw["dK"], dw["P"])
     q, k, v = make_qkv(dw["B"], dw["H"], dw["N"], dw["dK"], dw["dV"],
                        seed=20261205 + 100 + 1000 * rank, dtype="bf16")
     dstate = torch.empty(dw["B"], dw["H"], dm, dw["dV"] + 1, device=dev)
     dout = torch.empty(dw["B"], dw["H"], w["dV"], device=dev)
-    sata.sata_prefill(q.to(dev), k.to(dev), v.to(dev), torch.empty(dw["B"], dw["H"], dw["N"], dw["dV"], device=dev),
+    sata.sata_prefill(q.to(dev), k.to(dev), v.to(dev),
+                      torch.empty(dw["B"], dw["H"], dw["N"], dw["dV"], device=dev),
                       dstate, dw["B"], dw["H"], dw["N"], dw["dK"], dw["dV"], dw["P"],
                       torch.bfloat16, stream)
+    m_lo = sata.sata_state_fp32_rows(dw["dK"], dw["P"])
+    lo = torch.empty(dw["B"], dw["H"], m_lo, dw["dV"] + 1, device=dev)
+    hi = torch.empty(dw["B"], dw["H"], dm - m_lo, dw["dV"] + 1, device=dev, dtype=torch.float16)
+    sata.sata_state_split(dstate, lo, hi, dw["B"], dw["H"], dw["dK"], dw["dV"], dw["P"], stream)
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
-    ds = DecodeStream(5)
     nsteps = args.decode_steps
+    ds = DecodeStream(5)
     toks = [tuple(t.to(dev) for t in ds.next()) for _ in range(args.warmup + nsteps)]
-    for i in range(args.warmup):
-        qt, kt, vt = toks[i]
-        sata.sata_decode_step(qt, kt, vt, dstate, dout, dw["B"], dw["H"], dw["dK"], dw["dV"],
-                              dw["P"], torch.bfloat16, stream)
-    torch.cuda.synchronize()
-    sata.sata_profile_enable(True)
-    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(nsteps)]
-    dk = {}
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(nsteps):
-        qt, kt, vt = toks[args.warmup + i]
-        dev_ev[i][0].record(stream)
-        sata.sata_decode_step(qt, kt, vt, dstate, dout, dw["B"], dw["H"], dw["dK"], dw["dV"],
-                              dw["P"], torch.bfloat16, stream)
-        dev_ev[i][1].record(stream)
-        for name, ms in sata.sata_profile_read():
-            dk.setdefault(name, []).append(ms)
-            launches += 1
-    torch.cuda.synchronize()
-    barrier()
-    clocks = sampler.stop()
-    sata.sata_profile_enable(False)
-    dms = [a.elapsed_time(b) for a, b in dev_ev]
-    dtotal = max_over_ranks(sum(dms))
-    dvalue = weak_scaling_value(world, nsteps, dw["B"], dtotal)
-    dbytes = 2 * dw["B"] * dw["H"] * dm * (dw["dV"] + 1) * 4
-    dkern_ms = statistics.mean(dk["decode_stream"])
-    dach = dbytes / (dkern_ms / 1e3) / 1e9
-    q4 = max(1, nsteps // 4)
-    decode = {
-        "value": dvalue, "unit": "tokens/s", "ms_per_step": dtotal / nsteps,
-        "steps": nsteps, "context_start": dw["N"] + args.warmup,
-        "latency_ms_first_quarter_median": statistics.median(dms[:q4]),
-        "latency_ms_last_quarter_median": statistics.median(dms[-q4:]),
-        "roofline": {"bound": "hbm", "kernel": "decode_stream", "achieved": dach,
-                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dach / pk["hbm_gbs"],
-                     "traffic": traffic_record("decode_stream"),
-                     "peak_source": pk["source"], "kernel_ms": dkern_ms,
-                     "algorithmic_bytes_per_launch": dbytes},
-    }
-    # e2e decode: H2D of the step's q,k,v from pinned host, D2H of out
     hq = [tuple(t.pin_memory() for t in ds.next()) for _ in range(min(nsteps, 64))]
-    dout_h = torch.empty(dout.shape, pin_memory=True)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    qt, kt, vt = toks[0]
-    a.record(stream)
-    for qh_, kh_, vh_ in hq:
-        qt.copy_(qh_, non_blocking=True)
-        kt.copy_(kh_, non_blocking=True)
-        vt.copy_(vh_, non_blocking=True)
+
+    def fp32_step(qt, kt, vt):
         sata.sata_decode_step(qt, kt, vt, dstate, dout, dw["B"], dw["H"], dw["dK"], dw["dV"],
                               dw["P"], torch.bfloat16, stream)
-        dout_h.copy_(dout, non_blocking=True)
-    b.record(stream)
-    b.synchronize()
-    de2e = max_over_ranks(a.elapsed_time(b))
-    decode["e2e"] = {"value": world * len(hq) * dw["B"] / (de2e / 1e3), "unit": "tokens/s",
-                     "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hq[0]),
-                     "d2h_bytes_per_step": dout.numel() * 4}
+
+    def mixed_step(qt, kt, vt):
+        sata.sata_decode_step_mixed(qt, kt, vt, lo, hi, dout, dw["B"], dw["H"], dw["dK"],
+                                    dw["dV"], dw["P"], torch.bfloat16, stream)
+
+    def time_decode(step, state_bytes, label):
+        """All decode steps timed one by one (context grows by one token per
+        step), the library's kernels timed by its event hook."""
+        nonlocal launches
+        for i in range(args.warmup):
+            step(*toks[i])
+        torch.cuda.synchronize()
+        sata.sata_profile_enable(True)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(nsteps)]
+        kk = {}
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(nsteps):
+            ev[i][0].record(stream)
+            step(*toks[args.warmup + i])
+            ev[i][1].record(stream)
+            for name, ms in sata.sata_profile_read():
+                kk.setdefault(name, []).append(ms)
+                launches += 1
+        torch.cuda.synchronize()
+        barrier()
+        sata.sata_profile_enable(False)
+        dms = [a.elapsed_time(b) for a, b in ev]
+        total = max_over_ranks(sum(dms))
+        dbytes = 2 * dw["B"] * dw["H"] * state_bytes
+        kname = max(kk, key=lambda n: sum(kk[n]))
+        kms = statistics.mean(kk[kname])
+        ach = dbytes / (kms / 1e3) / 1e9
+        qn = max(1, nsteps // 4)
+        quarters = [statistics.median(dms[j * qn:(j + 1) * qn]) for j in range(4)
+                    if dms[j * qn:(j + 1) * qn]]
+        res = {
+            "state": label, "value": weak_scaling_value(world, nsteps, dw["B"], total),
+            "unit": "tokens/s", "ms_per_step": total / nsteps, "steps": nsteps,
+            "context": [dw["N"] + args.warmup + 1, dw["N"] + args.warmup + nsteps],
+            "latency_ms_quarter_medians": quarters,
+            "latency_ms_min": min(dms), "latency_ms_max": max(dms),
+            "latency_flatness": max(quarters) / min(quarters) - 1.0,
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": ach,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+                         "traffic": traffic_record(kname),
+                         "peak_source": pk["source"], "kernel_ms": kms,
+                         "algorithmic_bytes_per_launch": dbytes},
+        }
+        # e2e: H2D of the step's q,k,v from pinned host memory, D2H of out
+        dout_h = torch.empty(dout.shape, pin_memory=True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        qt, kt, vt = toks[0]
+        a.record(stream)
+        for qh_, kh_, vh_ in hq:
+            qt.copy_(qh_, non_blocking=True)
+            kt.copy_(kh_, non_blocking=True)
+            vt.copy_(vh_, non_blocking=True)
+            step(qt, kt, vt)
+            dout_h.copy_(dout, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b))
+        res["e2e"] = {"value": world * len(hq) * dw["B"] / (e2e_ms / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hq[0]),
+                      "d2h_bytes_per_step": dout.numel() * 4}
+        return res
+
+    decode = time_decode(fp32_step, dm * (dw["dV"] + 1) * 4, "fp32")
+    decode["mixed_state"] = time_decode(
+        mixed_step, m_lo * (dw["dV"] + 1) * 4 + (dm - m_lo) * (dw["dV"] + 1) * 2,
+        f"rows of degree <= 2 fp32 ({m_lo}/head), degree 3 fp16 ({dm - m_lo}/head)")
+    clocks = sampler.stop()
     assert sata.sata_get_error() == sata.SATA_OK
 
     line = {
@@ -450,7 +473,8 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic: seeded i.i.d. N(0,1) q,k,v cast to bf16",
         "config": {"workload": WORKLOAD, "global_batch": world * PREFILL["B"] * PREFILL["H"],
                    "seq_len": PREFILL["N"], "parallelism": f"dp{world} (independent heads)",
-                   "l2": "prefill: 256 MiB L2 flush between timed steps; decode: 3.19 GB state > L2",
+                   "l2": "prefill: 256 MiB L2 flush between timed steps; decode: 3.19 GB fp32 "
+                         "(1.66 GB mixed) state > L2",
                    "decode_steps": nsteps},
         "roofline": roof, "decode": decode, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks,
@@ -535,7 +559,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--decode-steps", type=int, default=128)
+    ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--ref-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=["decode", "prefill", "prefill_full"], default=None,

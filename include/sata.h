@@ -130,6 +130,48 @@ int sata_decode_step(const void *q, const void *k, const void *v, float *state,
                      float *out, int B, int H, int dK, int dV, int P,
                      sata_dtype dt, sata_stream_t stream);
 
+/* ---- Mixed-precision decode state ("硬件优化路径与当前局限": fp16 storage
+ * halves the state's bandwidth).  The state of every head is stored as two
+ * arrays: its first m_lo rows (every row of degree <= 2, m_lo =
+ * C(dK+2, 2) when P >= 3, else all m rows) in fp32, and the other
+ * m - m_lo rows (degree >= 3) in IEEE fp16:
+ *     state_lo  [B, H, m_lo,     dV+1]  float
+ *     state_hi  [B, H, m - m_lo, dV+1]  IEEE binary16 (uint16 storage)
+ * Row order inside each array is the fp32 state's (degree-major,
+ * lexicographic).  The low-degree rows keep fp32 because their entries grow
+ * with every token (row 0 counts the tokens): in fp16 their increments would
+ * be lost.  The higher-degree rows are rounded to nearest at every update. */
+
+/* Rows per head kept in fp32 (m_lo above), or -1 if dK < 1 or P < 1.
+ * Host only. */
+int64_t sata_state_fp32_rows(int dK, int P);
+
+/* Converts an fp32 state [B, H, m, dV+1] into the two arrays of the mixed
+ * state (fp16 rows rounded to nearest).  state_hi may be NULL when m_lo = m.
+ * Asynchronous on `stream`.  Returns SATA_OK, SATA_ERR_INVALID_ARG (null or
+ * misaligned pointer, overlapping arrays, bad size), SATA_ERR_UNSUPPORTED or
+ * SATA_ERR_CUDA. */
+int sata_state_split(const float *state, float *state_lo, void *state_hi,
+                     int B, int H, int dK, int dV, int P, sata_stream_t stream);
+
+/* The inverse: the two arrays back into one fp32 state (exact).  Same
+ * arguments and returns as sata_state_split. */
+int sata_state_join(const float *state_lo, const void *state_hi, float *state,
+                    int B, int H, int dK, int dV, int P, sata_stream_t stream);
+
+/* sata_decode_step on a mixed-precision state, updated in place: the same
+ * per-token procedure ("恒定计算成本的工程实现"), with each updated fp16
+ * entry rounded to nearest before it is stored and read out.  dV must be 32
+ * or 64 (else SATA_ERR_UNSUPPORTED); other arguments and layouts as
+ * sata_decode_step.  Returns SATA_OK, SATA_ERR_INVALID_ARG,
+ * SATA_ERR_UNSUPPORTED, SATA_ERR_NOMEM or SATA_ERR_CUDA; a device-side wait
+ * that gave up (reported by sata_get_error as SATA_ERR_TIMEOUT) leaves the
+ * state undefined. */
+int sata_decode_step_mixed(const void *q, const void *k, const void *v,
+                           float *state_lo, void *state_hi, float *out,
+                           int B, int H, int dK, int dV, int P, sata_dtype dt,
+                           sata_stream_t stream);
+
 /* sata_decode_step without any device allocation.  (The paper has no
  * counterpart: this is an interface for callers that cannot allocate device
  * memory: hosts whose caching allocator owns the whole GPU, serving loops
@@ -160,7 +202,7 @@ int sata_decode_step_noalloc(const void *q, const void *k, const void *v,
                              sata_stream_t stream);
 
 /* Test hook (no counterpart on the pages).  Bounds every wait of a role in
- * the tensor-core prefill kernels (a producer, the MMA issuer, an epilogue or
+ * the tensor-core prefill kernels and the bulk-copy decode kernel (a producer, the MMA issuer, an epilogue or
  * generator warp waiting for another role) to `cycles` SM clock cycles;
  * cycles <= 0 restores the default bound (about 2 s).  A wait that runs out
  * records SATA_ERR_TIMEOUT for sata_get_error, makes every role of its CTA

@@ -72,6 +72,14 @@ def lib() -> ctypes.CDLL:
     L.sata_profile_read.restype = i
     L.sata_kernel_name.argtypes = [i]
     L.sata_kernel_name.restype = ctypes.c_char_p
+    L.sata_state_fp32_rows.argtypes = [i, i]
+    L.sata_state_fp32_rows.restype = i64
+    L.sata_state_split.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
+    L.sata_state_split.restype = i
+    L.sata_state_join.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
+    L.sata_state_join.restype = i
+    L.sata_decode_step_mixed.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    L.sata_decode_step_mixed.restype = i
     L.sata_test_set_wait_limit.argtypes = [ctypes.c_longlong]
     L.sata_test_set_wait_limit.restype = ctypes.c_longlong
     _lib = L
@@ -153,6 +161,33 @@ def sata_decode_step_noalloc(q, k, v, state, out, B, H, dK, dV, P, dtype, stream
                                         dK, dV, P, _dtype_code(dtype), _stream(stream))
     if st != SATA_OK:
         raise SataError(st, "sata_decode_step_noalloc")
+
+
+def sata_state_fp32_rows(dK: int, P: int) -> int:
+    return int(lib().sata_state_fp32_rows(dK, P))
+
+
+def sata_state_split(state, state_lo, state_hi, B, H, dK, dV, P, stream=None) -> None:
+    st = lib().sata_state_split(_ptr(state), _ptr(state_lo), _ptr(state_hi), B, H, dK, dV, P,
+                                _stream(stream))
+    if st != SATA_OK:
+        raise SataError(st, "sata_state_split")
+
+
+def sata_state_join(state_lo, state_hi, state, B, H, dK, dV, P, stream=None) -> None:
+    st = lib().sata_state_join(_ptr(state_lo), _ptr(state_hi), _ptr(state), B, H, dK, dV, P,
+                               _stream(stream))
+    if st != SATA_OK:
+        raise SataError(st, "sata_state_join")
+
+
+def sata_decode_step_mixed(q, k, v, state_lo, state_hi, out, B, H, dK, dV, P, dtype,
+                           stream=None) -> None:
+    st = lib().sata_decode_step_mixed(_ptr(q), _ptr(k), _ptr(v), _ptr(state_lo), _ptr(state_hi),
+                                      _ptr(out), B, H, dK, dV, P, _dtype_code(dtype),
+                                      _stream(stream))
+    if st != SATA_OK:
+        raise SataError(st, "sata_decode_step_mixed")
 
 
 def sata_get_error(stream=None) -> int:
@@ -248,3 +283,51 @@ def decode_step(q, k, v, state, P: int, out=None, stream=None):
         out = torch.empty(B, H, dV, device=q.device, dtype=torch.float32)
     sata_decode_step(q, k, v, state, out, B, H, dK, dV, P, q.dtype, stream)
     return out
+
+
+def split_state(state, P: int, stream=None):
+    """fp32 state [B,H,m,dV+1] -> (state_lo fp32 [B,H,m_lo,dV+1], state_hi
+    fp16 [B,H,m-m_lo,dV+1]), the mixed-precision decode state."""
+    import torch
+
+    B, H, m, D1 = state.shape
+    dK = _dk_of(m, P)
+    m_lo = sata_state_fp32_rows(dK, P)
+    lo = torch.empty(B, H, m_lo, D1, device=state.device, dtype=torch.float32)
+    hi = torch.empty(B, H, m - m_lo, D1, device=state.device, dtype=torch.float16)
+    sata_state_split(state, lo, hi if m > m_lo else None, B, H, dK, D1 - 1, P, stream)
+    return lo, hi
+
+
+def join_state(state_lo, state_hi, P: int, dK: int, stream=None):
+    """The mixed-precision state back to one fp32 state [B,H,m,dV+1]."""
+    import torch
+
+    B, H, m_lo, D1 = state_lo.shape
+    m = sata_basis_size(dK, P)
+    state = torch.empty(B, H, m, D1, device=state_lo.device, dtype=torch.float32)
+    sata_state_join(state_lo, state_hi if m > m_lo else None, state, B, H, dK, D1 - 1, P, stream)
+    return state
+
+
+def decode_step_mixed(q, k, v, state_lo, state_hi, P: int, out=None, stream=None):
+    """One token per head on the mixed-precision state (updated in place)."""
+    import torch
+
+    _check_qkv(q, k, v)
+    B, H = q.shape[:2]
+    dK = q.shape[-1]
+    dV = v.shape[-1]
+    if out is None:
+        out = torch.empty(B, H, dV, device=q.device, dtype=torch.float32)
+    m = sata_basis_size(dK, P)
+    hi = state_hi if m > state_lo.shape[2] else None
+    sata_decode_step_mixed(q, k, v, state_lo, hi, out, B, H, dK, dV, P, q.dtype, stream)
+    return out
+
+
+def _dk_of(m: int, P: int) -> int:
+    for dK in (8, 16, 32, 64):
+        if sata_basis_size(dK, P) == m:
+            return dK
+    raise ValueError(f"no supported dK gives {m} basis rows at P={P}")

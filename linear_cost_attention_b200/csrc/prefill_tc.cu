@@ -688,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t out[32];
         if (ti < p.n_tiles) {
           const TileDesc td = sTiles[ti];
-          gen_tile(td, qrow, (uint32_t)(row & 7), p.W, out);
+          gen_tile<8>(td, qrow, (uint32_t)(row & 7), p.W, out);
         } else {
 #pragma unroll
           for (int q = 0; q < 32; ++q) out[q] = 0u;

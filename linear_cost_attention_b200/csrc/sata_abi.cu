@@ -266,6 +266,7 @@ extern "C" const char *sata_kernel_name(int id) {
     case K_TC_CHUNK_STATES: return "tc_chunk_states";
     case K_TC_READOUT: return "tc_readout";
     case K_TC_PREP: return "tc_prep";
+    case K_DECODE_BULK: return "decode_bulk";
   }
   return "unknown";
 }
@@ -349,8 +350,107 @@ extern "C" int sata_decode_step(const void *q, const void *k, const void *v, flo
   const DeviceBasis *basis = get_device_basis(dK, P, &st);
   if (!basis) return st;
   prof_call_begin();
+  if (bulk_decode_supported(dV))
+    return launch_decode_bulk(q, k, v, state, nullptr, B, H, dK, dV, (int)m, 0, dt == SATA_BF16,
+                              basis, out, (cudaStream_t)stream);
   return launch_decode(q, k, v, state, out, B, H, dK, dV, P, dt == SATA_BF16, basis,
                        (cudaStream_t)stream);
+}
+
+// ------------------------------------------------ mixed-precision decode state
+namespace {
+
+// Rows per head kept in fp32 in the mixed state: every row of degree <= 2.
+int64_t mixed_lo_rows(int dK, int P) { return count_basis(dK, P < 3 ? P : 3); }
+
+// Shared validation of the mixed-state calls; fills m, m_lo.
+int check_mixed(const float *lo, const void *hi, int B, int H, int dK, int dV, int P,
+                int64_t *m, int64_t *m_lo) {
+  if (!lo || !aligned16(lo) || !aligned16(hi)) return SATA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1) return SATA_ERR_INVALID_ARG;
+  if (!supported_dim(dK) || !supported_dim(dV) || P < 1 || P > kMaxP) return SATA_ERR_UNSUPPORTED;
+  *m = count_basis(dK, P);
+  *m_lo = mixed_lo_rows(dK, P);
+  if (*m > *m_lo && !hi) return SATA_ERR_INVALID_ARG;
+  const long long BH = (long long)B * H;
+  if (BH * *m * (dV + 1) >= (1LL << 40)) return SATA_ERR_INVALID_ARG;
+  if (BH * (dK > dV + 1 ? dK : dV + 1) >= (1LL << 31)) return SATA_ERR_INVALID_ARG;
+  const size_t nlo = (size_t)BH * *m_lo * (dV + 1) * 4, nhi = (size_t)BH * (*m - *m_lo) * (dV + 1) * 2;
+  if (hi && nhi && overlaps(lo, nlo, hi, nhi)) return SATA_ERR_INVALID_ARG;
+  return SATA_OK;
+}
+
+}  // namespace
+
+extern "C" int64_t sata_state_fp32_rows(int dK, int P) {
+  if (dK < 1 || P < 1) return -1;
+  return mixed_lo_rows(dK, P);
+}
+
+extern "C" int sata_state_split(const float *state, float *state_lo, void *state_hi, int B, int H,
+                                int dK, int dV, int P, sata_stream_t stream) {
+  int64_t m = 0, m_lo = 0;
+  if (!state || !aligned16(state)) return SATA_ERR_INVALID_ARG;
+  const int st = check_mixed(state_lo, state_hi, B, H, dK, dV, P, &m, &m_lo);
+  if (st != SATA_OK) return st;
+  const long long BH = (long long)B * H;
+  const size_t ns = (size_t)BH * m * (dV + 1) * 4, nlo = (size_t)BH * m_lo * (dV + 1) * 4,
+               nhi = (size_t)BH * (m - m_lo) * (dV + 1) * 2;
+  if (overlaps(state, ns, state_lo, nlo) || (nhi && overlaps(state, ns, state_hi, nhi)))
+    return SATA_ERR_INVALID_ARG;
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
+  return launch_state_convert(true, const_cast<float *>(state), state_lo, state_hi, BH, (int)m,
+                              (int)m_lo, dV + 1, (cudaStream_t)stream);
+}
+
+extern "C" int sata_state_join(const float *state_lo, const void *state_hi, float *state, int B,
+                               int H, int dK, int dV, int P, sata_stream_t stream) {
+  int64_t m = 0, m_lo = 0;
+  if (!state || !aligned16(state)) return SATA_ERR_INVALID_ARG;
+  const int st = check_mixed(state_lo, state_hi, B, H, dK, dV, P, &m, &m_lo);
+  if (st != SATA_OK) return st;
+  const long long BH = (long long)B * H;
+  const size_t ns = (size_t)BH * m * (dV + 1) * 4, nlo = (size_t)BH * m_lo * (dV + 1) * 4,
+               nhi = (size_t)BH * (m - m_lo) * (dV + 1) * 2;
+  if (overlaps(state, ns, state_lo, nlo) || (nhi && overlaps(state, ns, state_hi, nhi)))
+    return SATA_ERR_INVALID_ARG;
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);
+  return launch_state_convert(false, state, const_cast<float *>(state_lo),
+                              const_cast<void *>(state_hi), BH, (int)m, (int)m_lo, dV + 1,
+                              (cudaStream_t)stream);
+}
+
+extern "C" int sata_decode_step_mixed(const void *q, const void *k, const void *v, float *state_lo,
+                                      void *state_hi, float *out, int B, int H, int dK, int dV,
+                                      int P, sata_dtype dt, sata_stream_t stream) {
+  if (!q || !k || !v || !out) return SATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return SATA_ERR_INVALID_ARG;
+  if (dt != SATA_F32 && dt != SATA_BF16) return SATA_ERR_INVALID_ARG;
+  int64_t m = 0, m_lo = 0;
+  const int st0 = check_mixed(state_lo, state_hi, B, H, dK, dV, P, &m, &m_lo);
+  if (st0 != SATA_OK) return st0;
+  if (!bulk_decode_supported(dV)) return SATA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  const size_t es = dt == SATA_F32 ? 4 : 2;
+  const size_t nq = BH * dK * es, nv = BH * dV * es, no = BH * dV * 4;
+  const size_t nlo = (size_t)BH * m_lo * (dV + 1) * 4, nhi = (size_t)BH * (m - m_lo) * (dV + 1) * 2;
+  const void *ins[3] = {q, k, v};
+  const size_t nin[3] = {nq, nq, nv};
+  for (int i = 0; i < 3; ++i)
+    if (overlaps(out, no, ins[i], nin[i]) || overlaps(state_lo, nlo, ins[i], nin[i]) ||
+        (nhi && overlaps(state_hi, nhi, ins[i], nin[i])))
+      return SATA_ERR_INVALID_ARG;
+  if (overlaps(out, no, state_lo, nlo) || (nhi && overlaps(out, no, state_hi, nhi)))
+    return SATA_ERR_INVALID_ARG;
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);  // one call at a time
+  int st = SATA_OK;
+  const DeviceBasis *basis = get_device_basis(dK, P, &st);
+  if (!basis) return st;
+  prof_call_begin();
+  return launch_decode_bulk(q, k, v, state_lo, m > m_lo ? state_hi : nullptr, B, H, dK, dV,
+                            (int)m_lo, (int)(m - m_lo), dt == SATA_BF16, basis, out,
+                            (cudaStream_t)stream);
 }
 
 extern "C" int sata_get_error(sata_stream_t stream) {

@@ -81,6 +81,17 @@ int launch_decode(const void *q, const void *k, const void *v, float *state, flo
                   int B, int H, int dK, int dV, int P, bool bf16,
                   const DeviceBasis *basis, cudaStream_t stream);
 
+// Decode through shared memory with bulk async copies (dV = 32 or 64): lo holds
+// the first m_lo rows of every head in fp32, hi (IEEE fp16, may be null when
+// m_hi = 0) the other m_hi rows.  An fp32 state is lo with m_hi = 0.
+bool bulk_decode_supported(int dV);
+int launch_decode_bulk(const void *q, const void *k, const void *v, float *lo, void *hi, int B,
+                       int H, int dK, int dV, int m_lo, int m_hi, bool bf16,
+                       const DeviceBasis *basis, float *out, cudaStream_t stream);
+// fp32 state <-> mixed state (split: state -> lo, hi; join: lo, hi -> state).
+int launch_state_convert(bool split, float *state, float *lo, void *hi, long long BH, int m,
+                         int m_lo, int D1, cudaStream_t stream);
+
 // Decode with caller-supplied basis tables (packed as in DeviceBasis) and
 // partial-sum scratch y of at least B*H*(dV+1) floats.
 int launch_decode_scratch(const void *q, const void *k, const void *v, float *state, float *out,
@@ -96,6 +107,7 @@ enum KernelId {
   K_TC_CHUNK_STATES = 5,
   K_TC_READOUT = 6,
   K_TC_PREP = 7,
+  K_DECODE_BULK = 8,
 };
 void prof_call_begin();                          // start of an entry-point call
 void prof_kernel_begin(cudaStream_t s, int id);  // before a launch

@@ -1,10 +1,11 @@
 // Device-side generation of one 64-feature tile of the tile order
-// (tile_order.h) for one token, dK = 64.
+// (tile_order.h) for one token, dK = 8 G (G = 8 or 4 index octets).
 //
-// The token's bf16 row (64 elements) sits in shared memory as a 128-byte row
-// in the 128-byte-swizzled layout a TMA load produces: element i is in 16-byte
-// chunk i/8, stored at chunk position (i/8) ^ (row % 8).  The 64 outputs are
-// returned as 32 packed bf16x2 words in tile order.
+// The token's bf16 row sits in shared memory as a 128-byte row in the
+// 128-byte-swizzled layout a TMA load produces: element i is in 16-byte chunk
+// i/8, stored at chunk position (i/8) ^ (row % 8); for dK = 32 only chunks
+// 0..3 are read.  The 64 outputs are returned as 32 packed bf16x2 words in
+// tile order.
 //
 // Arithmetic (feature = w_alpha * prod x): OUTER and BC tiles form the pair
 // product u = w * x_i * x_j in fp32, round it to bf16 and multiply by the
@@ -28,9 +29,9 @@
 namespace sata {
 namespace tc {
 
-// Basis weights for dK = 64: 1/sqrt(alpha! * 64^(p/2)).
+// Basis weights 1/sqrt(alpha! * dK^(p/2)).
 struct GenWeights {
-  float w3, w3h;  // degree 3: alpha! = 1, 2  (64^-3/4 = 2^-4.5)
+  float w3, w3h;  // degree 3: alpha! = 1, 2
   float w3s;      // degree 3: alpha! = 6
   float w2, w2h;  // degree 2: alpha! = 1, 2
   float w1;       // degree 1
@@ -107,7 +108,8 @@ SATA_HD void gen_outer(const TileDesc &td, const uint8_t *row, uint32_t rsw,
   float ob[8];
   unpack8(load_chunk(row, rsw, td.o0), ob);
   const uint4 rc = load_chunk(row, rsw, td.o1);
-  const float s = (td.wsel == 0 ? W.w3 : W.w2) * (td.i1 < 64 ? load_elem(row, rsw, td.i1) : 1.f);
+  const float s =
+      (td.wsel == 0 ? W.w3 : W.w2) * (td.i1 != kNoIndex ? load_elem(row, rsw, td.i1) : 1.f);
 #pragma unroll
   for (int b = 0; b < 8; ++b) scale_chunk(s * ob[b], rc, &out[4 * b]);
 }
@@ -151,39 +153,40 @@ SATA_HD void gen_bc(const TileDesc &td, const uint8_t *row, uint32_t rsw,
 
 // ---- D: features 64*T + P of the concatenated in-octet triples; a tile
 // touches at most two octets, loaded once (ga = first, gb = second).
-template <int T> struct DOctets {
+template <int G, int T> struct DOctets {
   static constexpr int ga = (64 * T) / 120;
-  static constexpr int gb = (64 * T + 63) / 120 < 8 ? (64 * T + 63) / 120 : 7;
+  static constexpr int gb = (64 * T + 63) / 120 < G ? (64 * T + 63) / 120 : G - 1;
 };
 
-template <int T, int P>
+template <int G, int T, int P>
 SATA_HD float d_feature(const float (&xa)[8], const float (&xb)[8], const GenWeights &W) {
   constexpr int f = 64 * T + P;
-  if constexpr (f >= 120 * 8) {
+  if constexpr (f >= 120 * G) {
     return 0.f;
   } else {
     constexpr int g = f / 120, r = f % 120;
     constexpr int a = triple_at(r, 0), b = triple_at(r, 1), c = triple_at(r, 2);
     constexpr int fa = fact3(a, b, c);
     const float w = fa == 1 ? W.w3 : fa == 2 ? W.w3h : W.w3s;
-    const float(&x)[8] = (g == DOctets<T>::ga) ? xa : xb;
+    const float(&x)[8] = (g == DOctets<G, T>::ga) ? xa : xb;
     return w * x[a] * x[b] * x[c];
   }
 }
 
-template <int T, int... Q>
+template <int G, int T, int... Q>
 SATA_HD void d_variant(const uint8_t *row, uint32_t rsw, const GenWeights &W,
                        uint32_t (&out)[32], std::integer_sequence<int, Q...>) {
   float xa[8], xb[8];
-  unpack8(load_chunk(row, rsw, DOctets<T>::ga), xa);
-  unpack8(load_chunk(row, rsw, DOctets<T>::gb), xb);
-  ((out[Q] = pack2(d_feature<T, 2 * Q>(xa, xb, W), d_feature<T, 2 * Q + 1>(xa, xb, W))), ...);
+  unpack8(load_chunk(row, rsw, DOctets<G, T>::ga), xa);
+  unpack8(load_chunk(row, rsw, DOctets<G, T>::gb), xb);
+  ((out[Q] = pack2(d_feature<G, T, 2 * Q>(xa, xb, W), d_feature<G, T, 2 * Q + 1>(xa, xb, W))),
+   ...);
 }
 
 // ---- MISC: in-octet pairs (degree 2), degree 1, degree 0, padding.  The
 // octets a tile needs are loaded once into registers (mask of octets).
-template <int T> struct MiscOctets {
-  static constexpr int n2 = 36 * 8, n1 = 64;
+template <int G, int T> struct MiscOctets {
+  static constexpr int n2 = 36 * G, n1 = 8 * G;
   static constexpr int octet_of(int f) {
     return f < n2 ? f / 36 : (f < n2 + n1 ? (f - n2) / 8 : -1);
   }
@@ -197,10 +200,10 @@ template <int T> struct MiscOctets {
   }
 };
 
-template <int T, int P>
+template <int G, int T, int P>
 SATA_HD float misc_feature(const float (&xo)[8][8], const GenWeights &W) {
   constexpr int f = 64 * T + P;
-  constexpr int n2 = 36 * 8, n1 = 64;
+  constexpr int n2 = 36 * G, n1 = 8 * G;
   if constexpr (f < n2) {
     constexpr int g = f / 36, pr = f % 36;
     constexpr int a = pair_a(pr), b = pair_b(pr);
@@ -214,22 +217,52 @@ SATA_HD float misc_feature(const float (&xo)[8][8], const GenWeights &W) {
   }
 }
 
-template <int T, int... G>
+template <int G, int T, int... O>
 SATA_HD void misc_load(const uint8_t *row, uint32_t rsw, float (&xo)[8][8],
-                       std::integer_sequence<int, G...>) {
-  (((MiscOctets<T>::mask() >> G) & 1u ? unpack8(load_chunk(row, rsw, G), xo[G]) : void()), ...);
+                       std::integer_sequence<int, O...>) {
+  (((MiscOctets<G, T>::mask() >> O) & 1u ? unpack8(load_chunk(row, rsw, O), xo[O]) : void()),
+   ...);
 }
 
-template <int T, int... Q>
+template <int G, int T, int... Q>
 SATA_HD void misc_variant(const uint8_t *row, uint32_t rsw, const GenWeights &W,
                           uint32_t (&out)[32], std::integer_sequence<int, Q...>) {
   float xo[8][8];
-  misc_load<T>(row, rsw, xo, std::make_integer_sequence<int, 8>{});
-  ((out[Q] = pack2(misc_feature<T, 2 * Q>(xo, W), misc_feature<T, 2 * Q + 1>(xo, W))), ...);
+  misc_load<G, T>(row, rsw, xo, std::make_integer_sequence<int, G>{});
+  ((out[Q] = pack2(misc_feature<G, T, 2 * Q>(xo, W), misc_feature<G, T, 2 * Q + 1>(xo, W))),
+   ...);
+}
+
+// D and MISC tiles: variant v of the G-octet tile order (the switch keeps
+// every tile's indices compile-time constants).
+template <int G, int V = 0>
+SATA_HD void gen_d(int v, const uint8_t *row, uint32_t rsw, const GenWeights &W,
+                   uint32_t (&out)[32]) {
+  constexpr int nD = (120 * G + 63) / 64;
+  if constexpr (V < nD) {
+    if (v == V) {
+      d_variant<G, V>(row, rsw, W, out, std::make_integer_sequence<int, 32>{});
+      return;
+    }
+    gen_d<G, V + 1>(v, row, rsw, W, out);
+  }
+}
+template <int G, int V = 0>
+SATA_HD void gen_misc(int v, const uint8_t *row, uint32_t rsw, const GenWeights &W,
+                      uint32_t (&out)[32]) {
+  constexpr int nM = (36 * G + 8 * G + 1 + 63) / 64;
+  if constexpr (V < nM) {
+    if (v == V) {
+      misc_variant<G, V>(row, rsw, W, out, std::make_integer_sequence<int, 32>{});
+      return;
+    }
+    gen_misc<G, V + 1>(v, row, rsw, W, out);
+  }
 }
 
 // Generates tile td for the token whose swizzled row starts at `row`
-// (rsw = row index % 8 of that token inside its 8-row atom).
+// (rsw = row index % 8 of that token inside its 8-row atom); G = dK / 8.
+template <int G>
 SATA_HD void gen_tile(const TileDesc &td, const uint8_t *row, uint32_t rsw,
                                          const GenWeights &W, uint32_t (&out)[32]) {
   switch (td.type) {
@@ -248,37 +281,12 @@ SATA_HD void gen_tile(const TileDesc &td, const uint8_t *row, uint32_t rsw,
         case 7: gen_bc<7>(td, row, rsw, W, out); return;
         default: gen_bc<8>(td, row, rsw, W, out); return;
       }
-    case T_D: {
-      constexpr auto seq = std::make_integer_sequence<int, 32>{};
-      switch (td.variant) {
-        case 0: d_variant<0>(row, rsw, W, out, seq); return;
-        case 1: d_variant<1>(row, rsw, W, out, seq); return;
-        case 2: d_variant<2>(row, rsw, W, out, seq); return;
-        case 3: d_variant<3>(row, rsw, W, out, seq); return;
-        case 4: d_variant<4>(row, rsw, W, out, seq); return;
-        case 5: d_variant<5>(row, rsw, W, out, seq); return;
-        case 6: d_variant<6>(row, rsw, W, out, seq); return;
-        case 7: d_variant<7>(row, rsw, W, out, seq); return;
-        case 8: d_variant<8>(row, rsw, W, out, seq); return;
-        case 9: d_variant<9>(row, rsw, W, out, seq); return;
-        case 10: d_variant<10>(row, rsw, W, out, seq); return;
-        case 11: d_variant<11>(row, rsw, W, out, seq); return;
-        case 12: d_variant<12>(row, rsw, W, out, seq); return;
-        case 13: d_variant<13>(row, rsw, W, out, seq); return;
-        default: d_variant<14>(row, rsw, W, out, seq); return;
-      }
-    }
-    case T_MISC: {
-      constexpr auto seq = std::make_integer_sequence<int, 32>{};
-      switch (td.variant) {
-        case 0: misc_variant<0>(row, rsw, W, out, seq); return;
-        case 1: misc_variant<1>(row, rsw, W, out, seq); return;
-        case 2: misc_variant<2>(row, rsw, W, out, seq); return;
-        case 3: misc_variant<3>(row, rsw, W, out, seq); return;
-        case 4: misc_variant<4>(row, rsw, W, out, seq); return;
-        default: misc_variant<5>(row, rsw, W, out, seq); return;
-      }
-    }
+    case T_D:
+      gen_d<G>(td.variant, row, rsw, W, out);
+      return;
+    case T_MISC:
+      gen_misc<G>(td.variant, row, rsw, W, out);
+      return;
     default:
 #pragma unroll
       for (int i = 0; i < 32; ++i) out[i] = 0u;

@@ -30,7 +30,7 @@ Slot sorted2(int x, int y) { return {2, std::min(x, y), std::max(x, y), -1}; }
 }  // namespace
 
 bool build_tile_order(int dK, TileOrder *out) {
-  if (dK != 64) return false;
+  if (dK != 64 && dK != 32) return false;
   const int G = dK / 8;
   HostBasis hb = build_host_basis(dK, 4);
   std::map<uint32_t, int32_t> lex;
@@ -81,7 +81,7 @@ bool build_tile_order(int dK, TileOrder *out) {
     for (int h = g + 1; h < G; ++h) {
       for (int b = 0; b < 8; ++b)
         for (int c = 0; c < 8; ++c) s[8 * b + c] = sorted2(8 * g + b, 8 * h + c);
-      push({T_OUTER, 0, (uint8_t)dK, (uint8_t)g, (uint8_t)h, 0, 0, 1}, s);
+      push({T_OUTER, 0, kNoIndex, (uint8_t)g, (uint8_t)h, 0, 0, 1}, s);
     }
   // D: triples inside one octet
   const int nD = (120 * G + 63) / 64;

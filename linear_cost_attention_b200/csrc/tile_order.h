@@ -1,9 +1,10 @@
-// Tile order of the minimal basis for the tensor-core path (dK = 64, P = 4).
+// Tile order of the minimal basis for the tensor-core path (P = 4, dK = 64 or
+// 32).
 //
 // The basis rows (sorted index tuples, "对称张量分解的核心洞察") are regrouped
 // into tiles of 64 features whose structure is fixed, so that one thread per
 // token can generate a tile with compile-time register indices.  Indices are
-// split into octets g = i / 8 (8 octets for dK = 64):
+// split into G = dK / 8 octets g = i / 8:
 //
 //  OUTER  x[i1] * x[8*ga + b] * x[8*gb + c], b, c = 0..7 (64 features):
 //         degree 3 with three distinct octets gi < gj < gl (i1 = 8*gi + a;
@@ -14,10 +15,12 @@
 //         (g, g'); two such blocks fill 9 tiles (252 tiles).
 //  D      degree 3 inside one octet: the 120 triples a <= b <= c of each
 //         octet, concatenated over the 8 octets (15 tiles).
-//  MISC   degree 2 inside one octet (36 pairs per octet), degree 1 (64),
-//         degree 0 (1), zero padding (6 tiles).
-// 749 tiles = 47936 slots for the 47905 rows; 31 slots are zero padding.  Per
-// feature, the weight is the basis weight 1/sqrt(alpha! dK^(p/2)) of its row.
+//  MISC   degree 2 inside one octet (36 pairs per octet), degree 1 (dK),
+//         degree 0 (1), zero padding.
+// dK = 64: 749 tiles (448 OUTER-3, 252 BC, 28 OUTER-2, 15 D, 6 MISC) = 47936
+// slots for the 47905 rows.  dK = 32: 103 tiles (32, 54, 6, 8, 3) = 6592 slots
+// for the 6545 rows.  The other slots are zero padding.  Per feature, the
+// weight is the basis weight 1/sqrt(alpha! dK^(p/2)) of its row.
 #pragma once
 
 #include <stdint.h>
@@ -31,6 +34,7 @@ enum TileType : uint8_t { T_OUTER = 0, T_BC = 1, T_D = 2, T_MISC = 3, T_PAD = 4 
 struct TileDesc {  // 8 bytes; read by the generator warps
   uint8_t type, variant, i1, o0, o1, o2, o3, wsel;
 };
+constexpr uint8_t kNoIndex = 0xff;  // OUTER tile of degree 2: no first index
 
 // Index pairs a <= b and triples a <= b <= c inside one octet, lexicographic.
 __host__ __device__ constexpr int pair_a(int p) {
@@ -73,8 +77,8 @@ struct TileOrder {
   std::vector<int32_t> row_of_slot;  // [n_tiles*64] lexicographic basis row, -1 = padding
 };
 
-// Builds the tile order for dK = 64, P = 4 and checks that it covers every
-// basis row exactly once.  Returns false if the check fails.
+// Builds the tile order for dK = 64 or 32, P = 4, and checks that it covers
+// every basis row exactly once.  Returns false if the check fails.
 bool build_tile_order(int dK, TileOrder *out);
 
 }  // namespace sata

@@ -3,7 +3,8 @@
 // tests/test_tile_order_cpu.py with nvcc; needs no GPU.
 //   1. every basis row appears in exactly one tile slot;
 //   2. for random bf16 rows, every generated feature equals the basis weight
-//      times the product of its indexed entries, up to bf16 rounding.
+//      times the product of its indexed entries, up to bf16 rounding;
+// for dK = 64 (8 index octets) and dK = 32 (4 octets).
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -16,36 +17,42 @@
 
 using namespace sata;
 
-int main() {
+template <int G>
+int check(int dK, int want_tiles) {
   TileOrder to;
-  if (!build_tile_order(64, &to)) {
-    printf("FAIL build_tile_order\n");
+  if (!build_tile_order(dK, &to)) {
+    printf("FAIL build_tile_order dK=%d\n", dK);
     return 1;
   }
-  HostBasis hb = build_host_basis(64, 4);
-  printf("tiles %d slots %zu rows %lld\n", to.n_tiles, to.row_of_slot.size(), (long long)hb.m);
-  if (to.n_tiles != 749) {
+  HostBasis hb = build_host_basis(dK, 4);
+  printf("dK %d: tiles %d slots %zu rows %lld\n", dK, to.n_tiles, to.row_of_slot.size(),
+         (long long)hb.m);
+  if (to.n_tiles != want_tiles) {
     printf("FAIL tile count\n");
     return 1;
   }
+  // weights 1/sqrt(alpha! dK^(p/2)) by degree and multiplicity
+  const double d = dK;
   tc::GenWeights W;
-  W.w3 = (float)(1.0 / std::sqrt(512.0));
-  W.w3h = (float)(1.0 / std::sqrt(1024.0));
-  W.w3s = (float)(1.0 / std::sqrt(3072.0));
-  W.w2 = 0.125f;
-  W.w2h = (float)(1.0 / std::sqrt(128.0));
-  W.w1 = (float)(1.0 / std::sqrt(8.0));
-  std::mt19937 rng(1234);
+  W.w3 = (float)(1.0 / std::sqrt(std::pow(d, 1.5)));
+  W.w3h = (float)(1.0 / std::sqrt(2.0 * std::pow(d, 1.5)));
+  W.w3s = (float)(1.0 / std::sqrt(6.0 * std::pow(d, 1.5)));
+  W.w2 = (float)(1.0 / std::sqrt(d));
+  W.w2h = (float)(1.0 / std::sqrt(2.0 * d));
+  W.w1 = (float)(1.0 / std::sqrt(std::sqrt(d)));
+  std::mt19937 rng(1234 + dK);
   std::normal_distribution<float> nd(0.f, 1.f);
   double worst = 0;
   long bad = 0;
   for (int trial = 0; trial < 16; ++trial) {
-    // a token row in the 128-byte swizzled layout, at row index r (swizzle r % 8)
+    // a token row in the 128-byte swizzled layout, at row index r (swizzle r % 8);
+    // entries past dK are garbage that the generator must not read
     const uint32_t r = trial % 8;
     float x[64];
     uint16_t bits[64];
     for (int i = 0; i < 64; ++i) {
-      __nv_bfloat16 b = __float2bfloat16_rn(trial == 15 ? (float)(i % 7) - 3.f : nd(rng));
+      const float val = i >= dK ? 1e30f : (trial == 15 ? (float)(i % 7) - 3.f : nd(rng));
+      __nv_bfloat16 b = __float2bfloat16_rn(val);
       x[i] = __bfloat162float(b);
       memcpy(&bits[i], &b, 2);
     }
@@ -56,7 +63,7 @@ int main() {
     }
     for (int t = 0; t < to.n_tiles; ++t) {
       uint32_t out[32];
-      tc::gen_tile(to.tiles[t], row, r, W, out);
+      tc::gen_tile<G>(to.tiles[t], row, r, W, out);
       for (int p = 0; p < 64; ++p) {
         uint16_t h = (uint16_t)((out[p / 2] >> (16 * (p % 2))) & 0xffff);
         __nv_bfloat16 hbv;
@@ -72,7 +79,7 @@ int main() {
         const double tol = 3 * std::ldexp(1.0, -8) * std::fabs(ref) + 1e-30;
         if (row_id < 0 ? got != 0.f : err > tol) {
           if (bad < 10)
-            printf("mismatch tile %d type %d var %d slot %d row %d got %g ref %g\n", t,
+            printf("mismatch dK %d tile %d type %d var %d slot %d row %d got %g ref %g\n", dK, t,
                    to.tiles[t].type, to.tiles[t].variant, p, row_id, got, ref);
           ++bad;
         }
@@ -80,8 +87,13 @@ int main() {
       }
     }
   }
-  printf("worst relative %.3e bad %ld\n", worst, bad);
-  if (bad) {
+  printf("dK %d: worst relative %.3e bad %ld\n", dK, worst, bad);
+  return bad ? 1 : 0;
+}
+
+int main() {
+  int fails = check<8>(64, 749) + check<4>(32, 103);
+  if (fails) {
     printf("FAIL\n");
     return 1;
   }

@@ -151,3 +151,23 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(sata, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         sata.lib()
+
+
+def test_mixed_state_calls_rejected_on_host():
+    L = sata.lib()
+    A = 1 << 20
+    assert L.sata_state_fp32_rows(64, 4) == 2145 == math.comb(66, 2)
+    assert L.sata_state_fp32_rows(64, 2) == 65
+    assert L.sata_state_fp32_rows(0, 4) == -1
+    # hi array required when P >= 4 has fp16 rows
+    assert L.sata_state_split(A, 2 * A, None, 1, 1, 8, 8, 4, None) == sata.SATA_ERR_INVALID_ARG
+    assert L.sata_state_split(A, 2 * A + 8, 3 * A, 1, 1, 8, 8, 4, None) == sata.SATA_ERR_INVALID_ARG
+    assert L.sata_state_join(A, 3 * A, A, 1, 1, 8, 8, 4, None) == sata.SATA_ERR_INVALID_ARG
+    assert L.sata_state_split(A, 2 * A, 3 * A, 1, 1, 12, 8, 4, None) == sata.SATA_ERR_UNSUPPORTED
+    dm = L.sata_decode_step_mixed
+    assert dm(A, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 1, 1, 8, 16, 4, 1, None) == \
+        sata.SATA_ERR_UNSUPPORTED                                 # dV = 16: no bulk kernel
+    assert dm(A, 2 * A, 3 * A, 4 * A, None, 6 * A, 1, 1, 8, 32, 4, 1, None) == \
+        sata.SATA_ERR_INVALID_ARG                                 # missing fp16 array
+    assert dm(A, 2 * A, 3 * A, 4 * A, 5 * A, A, 1, 1, 8, 32, 4, 1, None) == \
+        sata.SATA_ERR_INVALID_ARG                                 # out aliases q
