@@ -87,10 +87,10 @@ int64_t sata_index_table(int dK, int p, int32_t *host_out, int64_t cap_elems);
 /* Causal prefill from a zero state.  Writes out (every token) and overwrites
  * state with S after the last token.  q, k, v, out, state: see layouts above;
  * out and state must not overlap each other or the inputs.
- * Paths: bf16 inputs with dK = dV = 64 and P = 4 run on the tcgen05 tensor
- * cores (features and chunk-boundary states rounded to bf16, in-chunk Taylor
- * scores split into bf16 hi + lo parts, fp32 accumulation); every other
- * supported case runs in fp32 on CUDA cores.  With the environment variable
+ * Paths: bf16 inputs with P = 4 and dK = dV = 64 or dK = dV = 32 run on the
+ * tcgen05 tensor cores (features and chunk-boundary states rounded to bf16,
+ * in-chunk Taylor scores split into bf16 hi + lo parts, fp32 accumulation);
+ * every other supported case runs in fp32 on CUDA cores.  With the environment variable
  * SATA_FORCE_SIMT=1 set before the first call, every prefill (and continued
  * prefill) takes the CUDA-core path, e.g. to cross-check the two paths.
  * Returns SATA_OK, SATA_ERR_INVALID_ARG, SATA_ERR_UNSUPPORTED, SATA_ERR_NOMEM

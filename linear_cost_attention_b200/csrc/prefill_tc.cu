@@ -1,33 +1,39 @@
-// Tensor-core (tcgen05) prefill for bf16 inputs with dK = dV = 64, P = 4.
+// Tensor-core (tcgen05) prefill for bf16 inputs with P = 4 and dK = dV = 64
+// or dK = dV = 32.
 //
 // Same chunked decomposition as the CUDA-core path (prefill_simt.cu), with
 // both state contractions on the 5th-generation tensor cores:
 //
-//   tc_transpose_kv  K, V [BH, N, 64] -> K^T, [V, 1]^T [BH, 65, Npad]: every
-//     basis monomial is a product of three K^T rows (row 64 = ones supplies the
-//     lower degrees) and [V, 1]^T is the K-major B operand of the state MMAs.
+//   tc_prep          K, V [BH, N, d] -> K^T [BH, dK+1, Npad], [V, 1]^T
+//     [BH, dV+1, Npad]: every basis monomial is a product of three K^T rows
+//     (row dK = ones supplies the lower degrees) and [V, 1]^T is the K-major B
+//     operand of the state MMAs and of the in-chunk P [V, 1] MMAs.  For
+//     dK = 32 it also writes Q and K padded to 64 columns with zeros, so that
+//     every tile keeps the 128-byte-swizzled layout of 64-element rows.
 //   tc_chunk_states  persistent CTAs (448 threads) over items = (head, two
-//     128-row state tiles); the tiles S'[128 x 80] (dV+1 = 65 columns padded
-//     to the MMA's N = 80) stay in TMEM for the whole sequence.  Per 128-token
-//     step: warp 0 brings the K^T and [V,1]^T boxes by TMA; warps 6-13 (one
-//     thread per basis row = TMEM lane) multiply three K^T rows for every
-//     token and store the unweighted monomials into a TMEM A stage; warp 1
-//     (one thread) issues 16 MMAs M = 128, N = 80, K = 16 (A from TMEM, B from
-//     shared memory), the two tiles alternating.  At each chunk boundary warps
-//     2-5 copy w^2 S' into a bf16 snapshot (the state before the next chunk,
-//     "恒定计算成本的工程实现": the fixed-size state); after the last token they
-//     write w S' as the fp32 state in lexicographic row order.  A continued
-//     prefill first loads S_0 / w into the tiles and S_0 w as snapshot 0.
-//   tc_readout       one CTA (512 threads) per (head, 128 tokens of chunk c):
-//     D[128 x 80] in TMEM accumulates phi(Q) S_(c-1) over 750 tiles of 64
+//     128-row state tiles); the tiles S'[128 x NP] (dV+1 columns padded to
+//     the MMA's N = NP, a multiple of 16) stay in TMEM for the whole sequence.
+//     Per 128-token step: warp 0 brings the K^T and [V,1]^T boxes by TMA;
+//     warps 6-13 (one thread per basis row = TMEM lane) multiply three K^T
+//     rows for every token and store the unweighted monomials into a TMEM A
+//     stage; warp 1 (one thread) issues 16 MMAs M = 128, N = NP, K = 16 (A
+//     from TMEM, B from shared memory), the two tiles alternating.  At each
+//     chunk boundary warps 2-5 copy w^2 S' into a bf16 snapshot (the state
+//     before the next chunk, "恒定计算成本的工程实现": the fixed-size state);
+//     after the last token they write w S' as the fp32 state in lexicographic
+//     row order.  A continued prefill first loads S_0 / w into the tiles and
+//     S_0 w as snapshot 0.
+//   tc_readout       one CTA (512 threads) per (head, 128 tokens), launched
+//     heaviest first (later chunks first, chunk 0 last):
+//     D[128 x NP] in TMEM accumulates phi(Q) S_(c-1) over the tiles of 64
 //     basis rows (warps 8-15, one thread per token = TMEM lane, generate the
 //     tiles' monomials into TMEM A stages; warp 0 streams the snapshot tiles by
 //     TMA) plus the in-chunk part sum_{c0 <= j <= i} T_4(s_ij) [v_j, 1] per
 //     64-key block: scores Q K^T into TMEM, T_4 and the causal mask by the
 //     epilogue warps 4-7, P split into bf16 hi + lo parts (T_4 rounded to bf16
 //     loses too much on rows whose denominator cancels), P_hi [V, 1] +
-//     P_lo [V, 1] into D; out = D[:, :64] / D[:, 64].  Warp 2 brings Q and the
-//     chunk's K, V blocks by TMA.
+//     P_lo [V, 1] into D; out = D[:, :dV] / D[:, dV].  Warp 2 brings Q and the
+//     chunk's K, [V, 1]^T blocks by TMA.
 //
 // The MMA-issuing thread waits on one barrier per stage: a wait there stalls
 // the tensor pipe, whose queue holds only a couple of MMAs.  Every mbarrier
@@ -48,38 +54,14 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 512;
-constexpr int kNP = 80;             // MMA N for [V, 1]: dV + 1 = 65 rounded up to 16
-constexpr uint32_t kRow = 128;      // bytes per 64-element bf16 row
-constexpr uint32_t kOne = 0x3F80u;  // bf16 1.0
+constexpr uint32_t kRow = 128;  // bytes per 64-element bf16 row (128-byte swizzle span)
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
   const uint32_t a = smem_u32(p);
   return p + (((a + 1023u) & ~1023u) - a);
 }
 
-// [V, 1] second column block: row r holds 1.0 at column 64 (logical chunk 0,
-// element 0), zeros elsewhere, in the 128-byte-swizzled layout.
-__device__ __forceinline__ void fill_ones(uint8_t *blk, int rows) {
-  for (int i = threadIdx.x; i < rows * 8; i += blockDim.x) {
-    const int r = i >> 3, c = i & 7;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (c == (r & 7)) v.x = kOne;
-    *reinterpret_cast<uint4 *>(blk + r * kRow + c * 16) = v;
-  }
-}
-
-// ============================================================ chunk states
-// One CTA per (head, kUF x 128 basis rows).  Thread = basis row = TMEM lane:
-// each generator thread forms its row's unweighted monomial x_i x_j x_l for
-// the step's tokens from the transposed keys (rows of K^T; index 64 is a row of
-// ones that is zero past the sequence end) and stores them with tcgen05.st
-// straight into the A operand in TMEM (basis rows x tokens, two tokens per
-// column).  The MMA accumulates S' += m(K)^T [V, 1] with [V, 1]^T as a K-major
-// B operand (rows of V^T plus its ones row; rows 65..79 are TMA zero fill).  The
-// basis weights are applied when S' leaves TMEM: state = w S', snapshot =
-// w^2 S' (the readout then multiplies by the unweighted m(q):
-// sum_a w_a m_a(q) w_a S'_a = phi(q) . S).
+// ------------------------------------------------------------ state kernel
 constexpr int kUF = 2;          // 128-row state tiles per item
 constexpr int kUT = 128;        // tokens per step
 constexpr int kUAS = 2;         // A stages (TMEM)
@@ -87,17 +69,48 @@ constexpr int kUKS = 4;         // K^T / V^T stages (shared memory)
 constexpr int kUGenWarps = 4 * kUF;
 constexpr int kUEpiWarp0 = 2, kUGenWarp0 = 6;  // warps 2..5 epilogue, 6.. generators
 constexpr int kUThreads = 32 * (kUGenWarp0 + kUGenWarps);
-constexpr int kMaxTiles = 768;  // tile table capacity in smem (readout)
-constexpr int kMaxDevices = 64;  // per-device launch attributes
-constexpr int kChunk = 4096;    // tokens per chunk (a multiple of the 128-token step)
-constexpr uint32_t kUColA = 160;               // TMEM: D at f*80, A from column 160
 constexpr uint32_t kUTmemCols = 512;
-constexpr uint32_t kUKTh = 9 * 1024;           // one 64-token K^T box: 65 rows x 128 B, padded
-constexpr uint32_t kUVTh = kNP * kRow;         // one 64-token [V,1]^T box: 80 rows x 128 B
-constexpr uint32_t kUKT = 2 * kUKTh, kUVT = 2 * kUVTh;  // per step (two boxes each)
-constexpr uint32_t kUOffKT = 0, kUOffVT = kUOffKT + kUKS * kUKT, kUOffBar = kUOffVT + kUKS * kUVT;
-constexpr uint32_t kUSmem = kUOffBar + 256 + 1024;
-static_assert(kUColA + kUAS * kUF * (kUT / 2) <= kUTmemCols && kUF * kNP <= kUColA, "TMEM budget");
+constexpr int kMaxDevices = 64;  // per-device launch attributes
+constexpr int kChunk = 4096;     // tokens per chunk (a multiple of the 128-token step)
+
+// ------------------------------------------------------------ readout
+constexpr int kThreads = 512;
+constexpr int kMaxTiles = 768;           // tile table capacity in smem
+constexpr int kRTS = 4;                  // feature tiles per pipeline stage
+constexpr int kRStages = 2;              // phi(Q) stages, in TMEM (32 columns per tile)
+constexpr int kRBS = 3;                  // snapshot stages (kRTS tiles each)
+constexpr int kKB = 64;                  // keys per in-chunk block
+constexpr uint32_t kRTile = 128 * kRow;  // 128 tokens x 64 features: 16 KiB
+constexpr uint32_t kRKB = kKB * kRow;    // 64 keys x 64 dims: 8 KiB
+constexpr uint32_t kRColS = 96, kRColA = 160;  // TMEM: D 0..NP-1, scores 96..159, A stages
+constexpr uint32_t kRTmemCols = 512;
+static_assert(kRColA + 32 * kRTS * kRStages <= kRTmemCols, "TMEM budget");
+
+// Shapes of one (dK, dV) instantiation.
+template <int DK, int DV> struct Tc {
+  static constexpr int D1 = DV + 1;                // [V, 1] columns
+  static constexpr int NP = (D1 + 15) / 16 * 16;   // MMA N (rows D1.. of B are zero fill)
+  static constexpr int KR = DK + 1;                // K^T rows, the last one all ones
+  static constexpr int G = DK / 8;                 // index octets of the tile order
+  static constexpr float kScale = DK == 64 ? 0.125f : 0.17677669529663687f;  // 1/sqrt(dK)
+  static_assert(DK == 64 || DK == 32, "the tile order exists for dK = 64 and 32");
+  static_assert(NP <= (int)kRColS, "D columns below the score columns");
+  // state kernel shared memory: K^T and [V,1]^T boxes of 64 tokens, two per step
+  static constexpr uint32_t UKTh = (KR * kRow + 1023) / 1024 * 1024;
+  static constexpr uint32_t UVTh = NP * kRow;
+  static constexpr uint32_t UKT = 2 * UKTh, UVT = 2 * UVTh;
+  static constexpr uint32_t UOffKT = 0, UOffVT = kUKS * UKT, UOffBar = UOffVT + kUKS * UVT;
+  static constexpr uint32_t USmem = UOffBar + 256 + 1024;
+  static constexpr uint32_t UColA = (kUF * NP + 31) / 32 * 32;  // TMEM: D at f*NP, A from here
+  static_assert(UColA + kUAS * kUF * (kUT / 2) <= kUTmemCols, "TMEM budget");
+  // readout shared memory
+  static constexpr uint32_t RB = NP * kRow;    // NP x 64 snapshot tile
+  static constexpr uint32_t RVT = NP * kRow;   // NP x 64-key [V,1]^T block
+  static constexpr uint32_t ROffQ = 0, ROffB = ROffQ + kRTile, ROffK = ROffB + kRBS * kRTS * RB,
+                            ROffVT = ROffK + kRKB, ROffP = ROffVT + RVT,
+                            ROffTiles = ROffP + 2 * kRTile, ROffBar = ROffTiles + kMaxTiles * 8;
+  static constexpr uint32_t RSmem = ROffBar + 512 + 1024;  // barriers, TMEM slot, flag
+};
 
 // TMEM lane -> slot inside a 128-row state tile.  Within each 32-lane warp
 // quarter, lane 4c + b holds slot 8b + c: in the 8 x 8 tiles (index octets b, c)
@@ -109,25 +122,38 @@ __host__ __device__ constexpr int lane_slot(int r) {
 }
 
 struct UParams {
-  const uint32_t *slot_idx;  // [m_pad] i | j << 8 | l << 16 (64 = the ones row)
+  const uint32_t *slot_idx;  // [m_pad] i | j << 8 | l << 16 (dK = the ones row)
   const float *slot_w;       // [m_pad] basis weight (0 on padding)
   const int32_t *row_of_slot;
   int n_mt;                  // 128-row tiles (m_pad / 128)
   int N, C, nsnap, m, m_pad, n_batches, n_items, head0;
   int cont;             // 1: start from the state in `state` (continued prefill)
-  __nv_bfloat16 *snap;  // [G][nsnap][65][m_pad]; slot 0 = initial state if cont
-  float *state;         // [BH][m][65]
+  __nv_bfloat16 *snap;  // [G][nsnap][dV+1][m_pad]; slot 0 = initial state if cont
+  float *state;         // [BH][m][dV+1]
   int *err;
   long long wait_limit;  // cycles before a role's wait gives up (drains: full limit)
 };
 
+// One CTA per (head, kUF x 128 basis rows).  Thread = basis row = TMEM lane:
+// each generator thread forms its row's unweighted monomial x_i x_j x_l for
+// the step's tokens from the transposed keys (rows of K^T; index dK is a row of
+// ones that is zero past the sequence end) and stores them with tcgen05.st
+// straight into the A operand in TMEM (basis rows x tokens, two tokens per
+// column).  The MMA accumulates S' += m(K)^T [V, 1] with [V, 1]^T as a K-major
+// B operand (rows of V^T plus its ones row; rows dV+1.. are TMA zero fill).
+// The basis weights are applied when S' leaves TMEM: state = w S', snapshot =
+// w^2 S' (the readout then multiplies by the unweighted m(q):
+// sum_a w_a m_a(q) w_a S'_a = phi(q) . S).
+template <int DK, int DV>
 __global__ void __launch_bounds__(kUThreads, 1)
     tc_chunk_states(const __grid_constant__ CUtensorMap tmKT, const __grid_constant__ CUtensorMap tmVT,
                     const UParams p) {
+  using S = Tc<DK, DV>;
+  constexpr int D1 = S::D1, NP = S::NP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sKT = smem + kUOffKT, *sVT = smem + kUOffVT;
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kUOffBar);
+  uint8_t *sKT = smem + S::UOffKT, *sVT = smem + S::UOffVT;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S::UOffBar);
   uint64_t *kv_full = bar, *kv_empty = bar + kUKS, *a_full = bar + 2 * kUKS,
            *a_empty = a_full + kUAS, *snap_full = a_empty + kUAS, *snap_done = snap_full + kUF,
            *drain = snap_done + kUF, *d_ready = drain + 1;
@@ -167,7 +193,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
   };
 
   if (warp == 0) {
-    // ---------------- TMA producer: K^T (65 rows) and [V,1]^T (80 rows), 2 x 64 tokens
+    // ---------------- TMA producer: K^T (dK+1 rows) and [V,1]^T (NP rows), 2 x 64 tokens
     if (lane == 0) {
       prefetch_tensormap(&tmKT);
       prefetch_tensormap(&tmVT);
@@ -177,13 +203,15 @@ __global__ void __launch_bounds__(kUThreads, 1)
         const int hb = item / p.n_batches;
         for (int s = 0; s < nsub; ++s, ++it) {
           const int st = it % kUKS;
-          if (it >= kUKS &&
-              !(ok = mbar_wait(&kv_empty[st], ((it / kUKS) - 1) & 1, abort_flag, p.err, p.wait_limit)))
+          if (it >= kUKS && !(ok = mbar_wait(&kv_empty[st], ((it / kUKS) - 1) & 1, abort_flag,
+                                             p.err, p.wait_limit)))
             break;
-          mbar_arrive_expect_tx(&kv_full[st], 2 * 65 * kRow + 2 * kUVTh);
+          mbar_arrive_expect_tx(&kv_full[st], 2 * S::KR * kRow + 2 * S::UVTh);
           for (int h = 0; h < 2; ++h) {
-            tma_load_3d(sKT + st * kUKT + h * kUKTh, &tmKT, &kv_full[st], s * kUT + 64 * h, 0, hb);
-            tma_load_3d(sVT + st * kUVT + h * kUVTh, &tmVT, &kv_full[st], s * kUT + 64 * h, 0, hb);
+            tma_load_3d(sKT + st * S::UKT + h * S::UKTh, &tmKT, &kv_full[st], s * kUT + 64 * h, 0,
+                        hb);
+            tma_load_3d(sVT + st * S::UVT + h * S::UVTh, &tmVT, &kv_full[st], s * kUT + 64 * h, 0,
+                        hb);
           }
         }
       }
@@ -195,7 +223,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, kNP, false, false);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, NP, false, false);
       uint32_t it = 0, events = 0, items = 0;
       bool after_event = false;
       bool ok = true;
@@ -211,9 +239,10 @@ __global__ void __launch_bounds__(kUThreads, 1)
           // a_full also covers kv_full: every generator warp waited on kv_full[ks]
           // before arriving.  One barrier wait per step: a wait in this thread
           // stalls until the MMAs already issued have drained.
-          if (!(ok = mbar_wait(&a_full[as], (it / kUAS) & 1, abort_flag, p.err, p.wait_limit))) break;
+          if (!(ok = mbar_wait(&a_full[as], (it / kUAS) & 1, abort_flag, p.err, p.wait_limit)))
+            break;
           tc_fence_after();
-          const uint32_t b0 = smem_u32(sVT + ks * kUVT);
+          const uint32_t b0 = smem_u32(sVT + ks * S::UVT);
           const bool event = is_event(s);
           if (after_event) {
             // every tile's barrier is waited once per event, in order, so no
@@ -227,11 +256,11 @@ __global__ void __launch_bounds__(kUThreads, 1)
           // different TMEM columns and do not wait for each other
 #pragma unroll
           for (int k = 0; k < kUT / 16; ++k) {
-            const uint64_t bd = smem_desc_sw128(b0 + (k >> 2) * kUVTh + 32 * (k & 3), 16, 1024);
+            const uint64_t bd = smem_desc_sw128(b0 + (k >> 2) * S::UVTh + 32 * (k & 3), 16, 1024);
 #pragma unroll
             for (int f = 0; f < kUF; ++f)
               if (f < nmt)
-                mma_bf16_ts(tmem + f * kNP, tmem + kUColA + (as * kUF + f) * (kUT / 2) + 8 * k, bd,
+                mma_bf16_ts(tmem + f * NP, tmem + S::UColA + (as * kUF + f) * (kUT / 2) + 8 * k, bd,
                             idesc, (s > 0 || k > 0 || p.cont) ? 1u : 0u);
           }
           after_event = false;
@@ -268,18 +297,18 @@ __global__ void __launch_bounds__(kUThreads, 1)
           const int slot = mt * 128 + lane_slot(row);
           const float w = p.slot_w[slot];
           const int r = p.row_of_slot[slot];
-          const float *src = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * 65;
-          __nv_bfloat16 *sdst = p.snap + ((size_t)hb * p.nsnap * 65) * p.m_pad + slot;
-          uint32_t v[kNP];
+          const float *src = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * D1;
+          __nv_bfloat16 *sdst = p.snap + ((size_t)hb * p.nsnap * D1) * p.m_pad + slot;
+          uint32_t v[NP];
 #pragma unroll
-          for (int n = 0; n < kNP; ++n) {
-            const float x = (n < 65 && r >= 0) ? src[n] : 0.f;
+          for (int n = 0; n < NP; ++n) {
+            const float x = (n < D1 && r >= 0) ? src[n] : 0.f;
             v[n] = __float_as_uint(w != 0.f ? x / w : 0.f);
-            if (n < 65) sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(w * x);
+            if (n < D1) sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(w * x);
           }
 #pragma unroll
-          for (int j = 0; j < kNP / 16; ++j)
-            tmem_st16(tmem + tl + f * kNP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+          for (int j = 0; j < NP / 16; ++j)
+            tmem_st16(tmem + tl + f * NP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
         }
         tmem_st_wait();
         tc_fence_before();
@@ -298,14 +327,14 @@ __global__ void __launch_bounds__(kUThreads, 1)
           const int slot = mt * 128 + lane_slot(row);
           const float w = live ? p.slot_w[slot] : 0.f;
           const int r = (live && !boundary) ? p.row_of_slot[slot] : -1;
-          __nv_bfloat16 *sdst = p.snap + ((size_t)(hb * p.nsnap + c) * 65) * p.m_pad + slot;
-          float *tdst = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * 65;
+          __nv_bfloat16 *sdst = p.snap + ((size_t)(hb * p.nsnap + c) * D1) * p.m_pad + slot;
+          float *tdst = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * D1;
           const float scale = boundary ? w * w : w;
-          uint32_t v[kNP];
+          uint32_t v[NP];
           if (live) {
 #pragma unroll
-            for (int j = 0; j < kNP / 16; ++j)
-              tmem_ld16(tmem + tl + f * kNP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+            for (int j = 0; j < NP / 16; ++j)
+              tmem_ld16(tmem + tl + f * NP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
             tmem_ld_wait();
           }
           tc_fence_before();
@@ -314,11 +343,11 @@ __global__ void __launch_bounds__(kUThreads, 1)
           if (!live) continue;
           if (boundary) {
 #pragma unroll
-            for (int n = 0; n < 65; ++n)
+            for (int n = 0; n < D1; ++n)
               sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(scale * __uint_as_float(v[n]));
           } else if (r >= 0) {
 #pragma unroll
-            for (int n = 0; n < 65; ++n) tdst[n] = scale * __uint_as_float(v[n]);
+            for (int n = 0; n < D1; ++n) tdst[n] = scale * __uint_as_float(v[n]);
           }
         }
         ++events;
@@ -331,21 +360,25 @@ __global__ void __launch_bounds__(kUThreads, 1)
     const int q4 = warp & 3;            // TMEM lane quarter
     const int row = 32 * q4 + lane;     // basis row inside the tile
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
+    constexpr uint32_t kOnes = (uint32_t)DK * 0x10101u;  // three "ones" rows
     uint32_t it = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
       const int batch = item % p.n_batches;
       const int mt = batch * kUF + f;
-      uint32_t ix = 0x404040u;  // three "ones" rows
+      uint32_t ix = kOnes;
       if (mt < p.n_mt) ix = p.slot_idx[mt * 128 + lane_slot(row)];
       const uint32_t ri = (ix & 0xff) * kRow, rj = ((ix >> 8) & 0xff) * kRow,
                      rl = ((ix >> 16) & 0xff) * kRow;
       const uint32_t si = (ix & 7), sj = ((ix >> 8) & 7), sl = ((ix >> 16) & 7);
       for (int s = 0; ok && s < nsub; ++s, ++it) {
         const int ks = it % kUKS, as = it % kUAS;
-        if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err, p.wait_limit))) break;
+        if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err, p.wait_limit)))
+          break;
         if (it >= kUAS) {
-          if (!(ok = mbar_wait(&a_empty[as], ((it / kUAS) - 1) & 1, abort_flag, p.err, p.wait_limit))) break;
+          if (!(ok = mbar_wait(&a_empty[as], ((it / kUAS) - 1) & 1, abort_flag, p.err,
+                               p.wait_limit)))
+            break;
           // the MMAs of step it - kUAS are complete and this warp read its K^T
           // rows long ago: release that step's K^T / V^T stage
           __syncwarp();
@@ -353,7 +386,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
         }
 #pragma unroll 1
         for (int h = 0; h < kUT / 64; ++h) {  // 64 tokens (one K^T box) at a time
-          const uint32_t kt = smem_u32(sKT) + ks * kUKT + h * kUKTh;
+          const uint32_t kt = smem_u32(sKT) + ks * S::UKT + h * S::UKTh;
           uint32_t out[32];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -365,7 +398,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
             out[4 * c + 2] = bmul2(bmul2(xi.z, xj.z), xl.z);
             out[4 * c + 3] = bmul2(bmul2(xi.w, xj.w), xl.w);
           }
-          tmem_st32(tmem + tl + kUColA + (as * kUF + f) * (kUT / 2) + 32 * h, out);
+          tmem_st32(tmem + tl + S::UColA + (as * kUF + f) * (kUT / 2) + 32 * h, out);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -381,57 +414,63 @@ __global__ void __launch_bounds__(kUThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kUTmemCols);
 }
 
-// K [BH, N, 64] -> K^T [BH, 65, Npad] and V [BH, N, 64] -> V^T [BH, 65, Npad]:
-// rows 0..63 transposed, row 64 ones for t < N, zeros on the padding.
-__global__ void __launch_bounds__(256) tc_transpose_kv(const __nv_bfloat16 *__restrict__ k,
-                                                       const __nv_bfloat16 *__restrict__ v,
-                                                       __nv_bfloat16 *__restrict__ kt,
-                                                       __nv_bfloat16 *__restrict__ vt, int N,
-                                                       int Npad, int head0) {
+// Per group of heads: K [BH, N, dK] -> K^T [g, dK+1, Npad] and V [BH, N, dV]
+// -> [V,1]^T [g, dV+1, Npad] (rows transposed, the last row ones for t < N,
+// zeros on the padding); for dK < 64 also Q, K -> [g, Npad, 64] with zeros
+// past column dK and past token N.
+template <int DK, int DV>
+__global__ void __launch_bounds__(256) tc_prep(const __nv_bfloat16 *__restrict__ q,
+                                               const __nv_bfloat16 *__restrict__ k,
+                                               const __nv_bfloat16 *__restrict__ v,
+                                               __nv_bfloat16 *__restrict__ kt,
+                                               __nv_bfloat16 *__restrict__ vt,
+                                               __nv_bfloat16 *__restrict__ qpad,
+                                               __nv_bfloat16 *__restrict__ kpad, int N, int Npad,
+                                               int head0) {
   __shared__ __nv_bfloat16 tile[64][66];
   const int t0 = blockIdx.x * 64;
   const size_t bh = (size_t)head0 + blockIdx.y;
+  const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
   for (int which = 0; which < 2; ++which) {
+    const int d = which ? DV : DK;
     const __nv_bfloat16 *src = which ? v : k;
-    __nv_bfloat16 *dst = (which ? vt : kt) + (size_t)blockIdx.y * 65 * Npad;
+    __nv_bfloat16 *dst = (which ? vt : kt) + (size_t)blockIdx.y * (d + 1) * Npad;
     __syncthreads();
-    for (int e = threadIdx.x; e < 64 * 64; e += 256) {
-      const int t = e >> 6, d = e & 63;
-      tile[t][d] = (t0 + t < N) ? src[(bh * N + t0 + t) * 64 + d] : __float2bfloat16_rn(0.f);
+    for (int e = threadIdx.x; e < 64 * d; e += 256) {
+      const int t = e / d, c = e % d;
+      tile[t][c] = (t0 + t < N) ? src[(bh * N + t0 + t) * d + c] : zero;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < 65 * 64; e += 256) {
-      const int d = e >> 6, t = e & 63;
-      dst[(size_t)d * Npad + t0 + t] =
-          d < 64 ? tile[t][d] : __float2bfloat16_rn(t0 + t < N ? 1.f : 0.f);
+    for (int e = threadIdx.x; e < (d + 1) * 64; e += 256) {
+      const int c = e >> 6, t = e & 63;
+      dst[(size_t)c * Npad + t0 + t] =
+          c < d ? tile[t][c] : __float2bfloat16_rn(t0 + t < N ? 1.f : 0.f);
+    }
+  }
+  if constexpr (DK < 64) {
+    for (int which = 0; which < 2; ++which) {
+      const __nv_bfloat16 *src = which ? k : q;
+      __nv_bfloat16 *dst = (which ? kpad : qpad) + (size_t)blockIdx.y * Npad * 64;
+      for (int e = threadIdx.x; e < 64 * 64; e += 256) {
+        const int t = e >> 6, c = e & 63;
+        dst[(size_t)(t0 + t) * 64 + c] =
+            (c < DK && t0 + t < N) ? src[(bh * N + t0 + t) * DK + c] : zero;
+      }
     }
   }
 }
 
 // ============================================================ readout
-constexpr int kRTS = 4;                  // feature tiles per pipeline stage
-constexpr int kRStages = 2;              // phi(Q) stages, in TMEM (32 columns per tile)
-constexpr int kRBS = 3;                  // snapshot stages (kRTS tiles each)
-constexpr int kKB = 64;                  // keys per in-chunk block
-constexpr uint32_t kRTile = 128 * kRow;  // 128 tokens x 64 features: 16 KiB
-constexpr uint32_t kRB = kNP * kRow;     // 80 x 64 snapshot tile: 10 KiB
-constexpr uint32_t kRKV = kKB * kRow;    // 64 keys x 64: 8 KiB
-constexpr uint32_t kRColS = 96, kRColA = 160;  // TMEM: D 0..79, scores 96..159, A stages
-constexpr uint32_t kRTmemCols = 512;
-static_assert(kRColA + 32 * kRTS * kRStages <= kRTmemCols, "TMEM budget");
-constexpr uint32_t kROffQ = 0, kROffB = kROffQ + kRTile,
-                   kROffK = kROffB + kRBS * kRTS * kRB, kROffV = kROffK + kRKV,
-                   kROffOnes = kROffV + kRKV, kROffP = kROffOnes + kRKV,
-                   kROffTiles = kROffP + 2 * kRTile, kROffBar = kROffTiles + kMaxTiles * 8;
-constexpr uint32_t kRSmem = kROffBar + 512 + 1024;  // 50 barriers + TMEM slot + flag
-
 struct RParams {
   const TileDesc *tiles;
   GenWeights W;
   int n_tiles;
   int N, C, nsnap, head0;
-  int cont;    // 1: snapshot slot 0 holds the state before chunk 0
-  float *out;  // [BH][N][64]
+  int qk_head0;  // head of group head 0 in the Q / K tensor maps (head0 for the caller's
+                 // q, k; 0 for the padded per-group copies)
+  int nblk;      // 128-token blocks per head
+  int cont;      // 1: snapshot slot 0 holds the state before chunk 0
+  float *out;    // [BH][N][dV]
   int *err;
   long long wait_limit;  // cycles before a role's wait gives up (drains: full limit)
 };
@@ -440,16 +479,19 @@ __device__ __forceinline__ float taylor4(float s) {
   return fmaf(fmaf(fmaf(s, 1.0f / 6.0f, 0.5f), s, 1.0f), s, 1.0f);
 }
 
+template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_readout(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
+               const __grid_constant__ CUtensorMap tmVT, const __grid_constant__ CUtensorMap tmS,
                const RParams p) {
+  using S = Tc<DK, DV>;
+  constexpr int NP = S::NP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  uint8_t *sQ = smem + kROffQ, *sB = smem + kROffB, *sK = smem + kROffK,
-          *sV = smem + kROffV, *sOnes = smem + kROffOnes, *sP = smem + kROffP;
-  TileDesc *sTiles = reinterpret_cast<TileDesc *>(smem + kROffTiles);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kROffBar);
+  uint8_t *sQ = smem + S::ROffQ, *sB = smem + S::ROffB, *sK = smem + S::ROffK,
+          *sVT = smem + S::ROffVT, *sP = smem + S::ROffP;
+  TileDesc *sTiles = reinterpret_cast<TileDesc *>(smem + S::ROffTiles);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S::ROffBar);
   uint64_t *q_full = bar, *kv_full = bar + 1, *kv_empty = bar + 2, *s_full = bar + 3,
            *p_full = bar + 4, *o_full = bar + 5, *a_full = bar + 6, *a_empty = a_full + kRStages,
            *b_full = a_empty + kRStages, *b_empty = b_full + kRBS;
@@ -458,8 +500,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert((6 + 2 * kRStages + 2 * kRBS + 2) * 8 <= 512, "barrier region");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * 128;
-  const int hrel = blockIdx.y;
+  // heaviest first: the last 128-token blocks (in the last chunks, with the
+  // longest in-chunk part) start first, chunk 0 (no inter-chunk part) last
+  const int g_heads = gridDim.x / p.nblk;
+  const int tb = p.nblk - 1 - (int)blockIdx.x / g_heads;
+  const int hrel = (int)blockIdx.x % g_heads;
+  const int t0 = tb * 128;
   const int bh = p.head0 + hrel;
   const int chunk = t0 / p.C;
   const int c0 = chunk * p.C;
@@ -486,8 +532,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  fill_ones(sOnes, kKB);
-  fence_proxy_async_smem();
   if (warp == 1) tmem_alloc(tmem_slot, kRTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -496,19 +540,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tD = tmem, tS = tmem + kRColS;
 
   if (warp == 0) {
-    // ---------------- TMA producer: snapshot tiles S_(c-1)[80 x 64 rows]
+    // ---------------- TMA producer: snapshot tiles S_(c-1)[NP x 64 rows]
     if (lane == 0 && inter) {
       prefetch_tensormap(&tmS);
       const int n_stages = (p.n_tiles + kRTS - 1) / kRTS;
       int i = 0;
       for (; i < n_stages; ++i) {
         const int st = i % kRBS;
-        if (i >= kRBS && !mbar_wait(&b_empty[st], ((i / kRBS) - 1) & 1, abort_flag, p.err, p.wait_limit))
+        if (i >= kRBS &&
+            !mbar_wait(&b_empty[st], ((i / kRBS) - 1) & 1, abort_flag, p.err, p.wait_limit))
           break;
         const int nt = min(kRTS, p.n_tiles - kRTS * i);
-        mbar_arrive_expect_tx(&b_full[st], nt * kRB);
+        mbar_arrive_expect_tx(&b_full[st], nt * S::RB);
         for (int t = 0; t < nt; ++t)
-          tma_load_3d(sB + (st * kRTS + t) * kRB, &tmS, &b_full[st], 64 * (kRTS * i + t), 0,
+          tma_load_3d(sB + (st * kRTS + t) * S::RB, &tmS, &b_full[st], 64 * (kRTS * i + t), 0,
                       hrel * p.nsnap + chunk - 1 + p.cont);
       }
       for (int j = max(0, i - kRBS); j < i; ++j) {
@@ -517,19 +562,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 2) {
-    // ---------------- TMA producer: Q once, then K, V blocks of the chunk
+    // ---------------- TMA producer: Q once, then K, [V,1]^T blocks of the chunk
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
+      prefetch_tensormap(&tmVT);
+      const int qk_head = p.qk_head0 + hrel;
       mbar_arrive_expect_tx(q_full, kRTile);
-      tma_load_3d(sQ, &tmQ, q_full, 0, t0, bh);
+      tma_load_3d(sQ, &tmQ, q_full, 0, t0, qk_head);
       int kb = 0;
       for (; kb < nkb; ++kb) {
         if (kb > 0 && !mbar_wait(kv_empty, (kb - 1) & 1, abort_flag, p.err, p.wait_limit)) break;
-        mbar_arrive_expect_tx(kv_full, 2 * kRKV);
-        tma_load_3d(sK, &tmK, kv_full, 0, c0 + kKB * kb, bh);
-        tma_load_3d(sV, &tmV, kv_full, 0, c0 + kKB * kb, bh);
+        mbar_arrive_expect_tx(kv_full, kRKB + S::RVT);
+        tma_load_3d(sK, &tmK, kv_full, 0, c0 + kKB * kb, qk_head);
+        tma_load_3d(sVT, &tmVT, kv_full, c0 + kKB * kb, 0, hrel);
       }
       volatile int never = 0;
       mbar_wait(q_full, 0, &never, p.err);
@@ -538,13 +584,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t id_inter = idesc_bf16_f32(128, kNP, false, false);
+      constexpr uint32_t id_nv = idesc_bf16_f32(128, NP, false, false);  // B: NP rows, K-major
       constexpr uint32_t id_qk = idesc_bf16_f32(128, kKB, false, false);
-      constexpr uint32_t id_pv = idesc_bf16_f32(128, kNP, false, true);
       bool d_init = false, ok = true;
       int kb_qk = 0, kb_pv = 0;
-      const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV);
-      const uint32_t p0 = smem_u32(sP), lbo_v = smem_u32(sOnes) - v0;
+      const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), vt0 = smem_u32(sVT);
+      const uint32_t p0 = smem_u32(sP);
       ok = mbar_wait(q_full, 0, abort_flag, p.err, p.wait_limit);
       // in-chunk part, advanced whenever its inputs are ready
       auto intra = [&](bool block) {
@@ -557,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < DK / 16; ++k)
               mma_bf16_ss(tS, smem_desc_sw128(q0 + 32 * k, 16, 1024),
                           smem_desc_sw128(k0 + 32 * k, 16, 1024), id_qk, k > 0 ? 1u : 0u);
             mma_commit(s_full);
@@ -572,9 +617,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 2 * (kKB / 16); ++k) {  // hi part, then lo part
               const int kk = k % (kKB / 16);
-              const uint64_t ad = smem_desc_sw128(p0 + (k / (kKB / 16)) * kRTile + 32 * kk, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(v0 + kk * 2048, lbo_v, 1024);
-              mma_bf16_ss(tD, ad, bd, id_pv, (d_init || k > 0) ? 1u : 0u);
+              const uint64_t ad =
+                  smem_desc_sw128(p0 + (k / (kKB / 16)) * kRTile + 32 * kk, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(vt0 + 32 * kk, 16, 1024);
+              mma_bf16_ss(tD, ad, bd, id_nv, (d_init || k > 0) ? 1u : 0u);
             }
             d_init = true;
             mma_commit(kv_empty);
@@ -590,15 +636,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = i % kRStages, bs = i % kRBS;
           // a_full also covers b_full: the generator warps wait on the snapshot
           // stage before arriving (one barrier wait per stage in this thread)
-          if (!(ok = mbar_wait(&a_full[st], (i / kRStages) & 1, abort_flag, p.err, p.wait_limit))) break;
+          if (!(ok = mbar_wait(&a_full[st], (i / kRStages) & 1, abort_flag, p.err, p.wait_limit)))
+            break;
           tc_fence_after();
           const int nt = min(kRTS, p.n_tiles - kRTS * i);
           for (int t = 0; t < nt; ++t) {
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               mma_bf16_ts(tD, tmem + kRColA + (st * kRTS + t) * 32 + 8 * k,
-                          smem_desc_sw128(b0 + (bs * kRTS + t) * kRB + 32 * k, 16, 1024),
-                          id_inter, (d_init || k > 0) ? 1u : 0u);
+                          smem_desc_sw128(b0 + (bs * kRTS + t) * S::RB + 32 * k, 16, 1024),
+                          id_nv, (d_init || k > 0) ? 1u : 0u);
             d_init = true;
           }
           mma_commit(&a_empty[st]);
@@ -635,13 +682,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < kKB / 2; ++j) {
           const int ka = key0 + 2 * j, kc = ka + 1;
-          const float ta = (ka <= tok && ka < p.N) ? taylor4(__uint_as_float(v[2 * j]) * 0.125f) : 0.f;
-          const float tb =
-              (kc <= tok && kc < p.N) ? taylor4(__uint_as_float(v[2 * j + 1]) * 0.125f) : 0.f;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(ta, tb);
+          const float ta =
+              (ka <= tok && ka < p.N) ? taylor4(__uint_as_float(v[2 * j]) * S::kScale) : 0.f;
+          const float tb2 =
+              (kc <= tok && kc < p.N) ? taylor4(__uint_as_float(v[2 * j + 1]) * S::kScale) : 0.f;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(ta, tb2);
           const float2 hf = __bfloat1622float2(h2);
           hi[j] = *reinterpret_cast<const uint32_t *>(&h2);
-          lo[j] = pack_bf16x2(ta - hf.x, tb - hf.y);
+          lo[j] = pack_bf16x2(ta - hf.x, tb2 - hf.y);
         }
         store_tile_row(sP, (uint32_t)row, hi);
         store_tile_row(sP + kRTile, (uint32_t)row, lo);
@@ -653,16 +701,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && (ok = mbar_wait(o_full, 0, abort_flag, p.err, p.wait_limit))) {
       tc_fence_after();
-      uint32_t v[kNP];
+      uint32_t v[NP];
 #pragma unroll
-      for (int j = 0; j < kNP / 16; ++j)
+      for (int j = 0; j < NP / 16; ++j)
         tmem_ld16(tD + tl + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
       tmem_ld_wait();
       if (tok < p.N) {
-        const float den = __uint_as_float(v[64]);
-        float4 *dst = reinterpret_cast<float4 *>(p.out + ((size_t)bh * p.N + tok) * 64);
+        const float den = __uint_as_float(v[DV]);
+        float4 *dst = reinterpret_cast<float4 *>(p.out + ((size_t)bh * p.N + tok) * DV);
 #pragma unroll
-        for (int n = 0; n < 16; ++n)
+        for (int n = 0; n < DV / 4; ++n)
           dst[n] = make_float4(__uint_as_float(v[4 * n]) / den, __uint_as_float(v[4 * n + 1]) / den,
                                __uint_as_float(v[4 * n + 2]) / den,
                                __uint_as_float(v[4 * n + 3]) / den);
@@ -688,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t out[32];
         if (ti < p.n_tiles) {
           const TileDesc td = sTiles[ti];
-          gen_tile<8>(td, qrow, (uint32_t)(row & 7), p.W, out);
+          gen_tile<S::G>(td, qrow, (uint32_t)(row & 7), p.W, out);
         } else {
 #pragma unroll
           for (int q = 0; q < 32; ++q) out[q] = 0u;
@@ -698,7 +746,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st32(tmem + ((uint32_t)(32 * (gw & 3)) << 16) + kRColA + (st * kRTS + t) * 32, out);
       }
       tmem_st_wait();
-      if (!(ok = mbar_wait(&b_full[i % kRBS], (i / kRBS) & 1, abort_flag, p.err, p.wait_limit))) break;
+      if (!(ok = mbar_wait(&b_full[i % kRBS], (i / kRBS) & 1, abort_flag, p.err, p.wait_limit)))
+        break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&a_full[st]);
@@ -744,16 +793,13 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-}  // namespace
-
-bool tc_supported(int dK, int dV, int P, bool bf16) {
-  return bf16 && dK == 64 && dV == 64 && P == 4;
-}
-
-int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, float *state,
-                      int B, int H, int N, bool cont, const DeviceBasis *basis, int *err,
-                      cudaStream_t stream) {
+template <int DK, int DV>
+int launch_tc(const void *q, const void *k, const void *v, float *out, float *state, int B,
+              int H, int N, bool cont, const DeviceBasis *basis, int *err, cudaStream_t stream) {
+  using S = Tc<DK, DV>;
+  constexpr int D1 = S::D1;
   const int BH = B * H;
   const int n_tiles = basis->n_tiles;  // even, padded
   if (n_tiles > kMaxTiles) return SATA_ERR_UNSUPPORTED;
@@ -767,21 +813,25 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
   // prefill) the initial state before chunk 0 in slot 0
   const int nsnap = (N + C - 1) / C - 1 + (cont ? 1 : 0);
   const int Npad = ((N + kUT - 1) / kUT) * kUT;  // multiple of the 128-token step
-  const size_t snap_head = (size_t)nsnap * 65 * m_pad * 2;
-  const size_t kt_head = (size_t)65 * Npad * 2;  // K^T or V^T of one head
-  const size_t per_head = snap_head + 2 * kt_head;
+  const size_t snap_head = (size_t)nsnap * D1 * m_pad * 2;
+  const size_t kt_head = (size_t)S::KR * Npad * 2, vt_head = (size_t)D1 * Npad * 2;
+  const size_t pad_head = DK < 64 ? (size_t)Npad * 64 * 2 : 0;  // padded Q or K of one head
+  const size_t per_head = snap_head + kt_head + vt_head + 2 * pad_head;
   const size_t budget = (size_t)4 << 30;
   const int G = (int)std::max<size_t>(1, std::min<size_t>(BH, budget / per_head));
   int st = SATA_OK;
-  uint8_t *ws = (uint8_t *)get_workspace(stream, per_head * G + 1024, &st);
+  uint8_t *ws = (uint8_t *)get_workspace(stream, per_head * G + 5 * 256, &st);
   if (!ws) return st;
-  const size_t kt_bytes = (kt_head * G + 255) & ~(size_t)255;
   __nv_bfloat16 *kt = reinterpret_cast<__nv_bfloat16 *>(ws);
-  __nv_bfloat16 *vt = reinterpret_cast<__nv_bfloat16 *>(ws + kt_bytes);
-  __nv_bfloat16 *snap = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * kt_bytes);
-  CUtensorMap mV64, mQ, mK64, mS, mKT, mVT;
-  if (!make_map(&mV64, v, 64, N, BH, 64) || !make_map(&mK64, k, 64, N, BH, 64) ||
-      !make_map(&mQ, q, 64, N, BH, 128))
+  uint8_t *p1 = ws + align256(kt_head * G);
+  __nv_bfloat16 *vt = reinterpret_cast<__nv_bfloat16 *>(p1);
+  uint8_t *p2 = p1 + align256(vt_head * G);
+  __nv_bfloat16 *qpad = reinterpret_cast<__nv_bfloat16 *>(p2);
+  uint8_t *p3 = p2 + align256(pad_head * G);
+  __nv_bfloat16 *kpad = reinterpret_cast<__nv_bfloat16 *>(p3);
+  __nv_bfloat16 *snap = reinterpret_cast<__nv_bfloat16 *>(p3 + align256(pad_head * G));
+  CUtensorMap mQ, mK, mS, mKT, mVT;
+  if (DK == 64 && (!make_map(&mQ, q, 64, N, BH, 128) || !make_map(&mK, k, 64, N, BH, kKB)))
     return SATA_ERR_CUDA;
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
@@ -791,10 +841,10 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
   static bool attr_done[kMaxDevices] = {};
   if (dev < 0 || dev >= kMaxDevices) return SATA_ERR_CUDA;
   if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(tc_chunk_states, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kUSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(tc_readout, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmem) !=
-            cudaSuccess)
+    if (cudaFuncSetAttribute(tc_chunk_states<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             S::USmem) != cudaSuccess ||
+        cudaFuncSetAttribute(tc_readout<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             S::RSmem) != cudaSuccess)
       return SATA_ERR_CUDA;
     attr_done[dev] = true;
   }
@@ -802,19 +852,23 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
 
   const int n_mt = m_pad / 128;
   const int n_batches = (n_mt + kUF - 1) / kUF;
+  const int nblk = (N + 127) / 128;
   GenWeights ones;  // the readout generates unweighted monomials
   ones.w3 = ones.w3h = ones.w3s = ones.w2 = ones.w2h = ones.w1 = 1.f;
   for (int h0 = 0; h0 < BH; h0 += G) {
     const int g = std::min(G, BH - h0);
-    if (!make_map(&mKT, kt, (uint64_t)Npad, 65, (uint64_t)g, 65) ||
-        !make_map(&mVT, vt, (uint64_t)Npad, 65, (uint64_t)g, kNP))
+    if (!make_map(&mKT, kt, (uint64_t)Npad, S::KR, (uint64_t)g, S::KR) ||
+        !make_map(&mVT, vt, (uint64_t)Npad, D1, (uint64_t)g, S::NP))
       return SATA_ERR_CUDA;
-    if (nsnap > 0 && !make_map(&mS, snap, (uint64_t)m_pad, 65, (uint64_t)g * nsnap, kNP))
+    if (DK < 64 && (!make_map(&mQ, qpad, 64, Npad, (uint64_t)g, 128) ||
+                    !make_map(&mK, kpad, 64, Npad, (uint64_t)g, kKB)))
+      return SATA_ERR_CUDA;
+    if (nsnap > 0 && !make_map(&mS, snap, (uint64_t)m_pad, D1, (uint64_t)g * nsnap, S::NP))
       return SATA_ERR_CUDA;
     prof_kernel_begin(stream, K_TC_PREP);
-    tc_transpose_kv<<<dim3(Npad / 64, g), 256, 0, stream>>>(
-        reinterpret_cast<const __nv_bfloat16 *>(k), reinterpret_cast<const __nv_bfloat16 *>(v),
-        kt, vt, N, Npad, h0);
+    tc_prep<DK, DV><<<dim3(Npad / 64, g), 256, 0, stream>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(q), reinterpret_cast<const __nv_bfloat16 *>(k),
+        reinterpret_cast<const __nv_bfloat16 *>(v), kt, vt, qpad, kpad, N, Npad, h0);
     prof_kernel_end(stream);
     UParams up;
     up.slot_idx = basis->slot_idx;
@@ -835,7 +889,8 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
     up.err = err;
     up.wait_limit = tc_wait_limit();
     prof_kernel_begin(stream, K_TC_CHUNK_STATES);
-    tc_chunk_states<<<std::min(up.n_items, nsm), kUThreads, kUSmem, stream>>>(mKT, mVT, up);
+    tc_chunk_states<DK, DV><<<std::min(up.n_items, nsm), kUThreads, S::USmem, stream>>>(mKT, mVT,
+                                                                                      up);
     prof_kernel_end(stream);
     RParams rp;
     rp.tiles = reinterpret_cast<const TileDesc *>(basis->tile_desc);
@@ -845,16 +900,34 @@ int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, f
     rp.C = C;
     rp.nsnap = nsnap;
     rp.head0 = h0;
+    rp.qk_head0 = DK == 64 ? h0 : 0;
+    rp.nblk = nblk;
     rp.cont = cont ? 1 : 0;
     rp.out = out;
     rp.err = err;
     rp.wait_limit = tc_wait_limit();
     if (nsnap == 0) mS = mQ;  // never read: no chunk has a predecessor
     prof_kernel_begin(stream, K_TC_READOUT);
-    tc_readout<<<dim3((N + 127) / 128, g), kThreads, kRSmem, stream>>>(mQ, mK64, mV64, mS, rp);
+    tc_readout<DK, DV><<<nblk * g, kThreads, S::RSmem, stream>>>(mQ, mK, mVT, mS, rp);
     prof_kernel_end(stream);
   }
   return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+bool tc_supported(int dK, int dV, int P, bool bf16) {
+  return bf16 && P == 4 && dK == dV && (dK == 64 || dK == 32);
+}
+
+int launch_prefill_tc(const void *q, const void *k, const void *v, float *out, float *state,
+                      int B, int H, int N, bool cont, const DeviceBasis *basis, int *err,
+                      cudaStream_t stream) {
+  if (basis->dK == 64)
+    return launch_tc<64, 64>(q, k, v, out, state, B, H, N, cont, basis, err, stream);
+  if (basis->dK == 32)
+    return launch_tc<32, 32>(q, k, v, out, state, B, H, N, cont, basis, err, stream);
+  return SATA_ERR_UNSUPPORTED;
 }
 
 }  // namespace sata

@@ -78,7 +78,7 @@ const DeviceBasis *get_device_basis(int dK, int P, int *status) {
                 cudaSuccess &&
             cudaMemcpy(db->w, w.data(), hb.m * sizeof(float), cudaMemcpyHostToDevice) ==
                 cudaSuccess;
-  if (ok && dK == 64 && P == 4) {
+  if (ok && (dK == 64 || dK == 32) && P == 4) {
     // tile order for the tensor-core path, padded to an even number of tiles
     TileOrder to;
     if (!build_tile_order(dK, &to)) {
@@ -93,16 +93,17 @@ const DeviceBasis *get_device_basis(int dK, int P, int *status) {
     }
     db->n_tiles = to.n_tiles;
     db->m_pad = (int64_t)to.n_tiles * 64;
-    // per slot: the row's index triple (unused slots point at row 64, the ones
+    // per slot: the row's index triple (unused slots point at row dK, the ones
     // row of the transposed keys) and its weight
-    std::vector<uint32_t> sidx(db->m_pad, 0x404040u);
+    const uint32_t ones3 = (uint32_t)dK * 0x10101u;
+    std::vector<uint32_t> sidx(db->m_pad, ones3);
     std::vector<float> sw(db->m_pad, 0.f);
     for (int64_t k = 0; k < db->m_pad; ++k) {
       const int32_t r = to.row_of_slot[k];
       if (r < 0) continue;
       uint32_t v = 0;
       for (int q = 0; q < 3; ++q) {
-        const int ii = q < hb.degree[r] ? hb.ix[4 * r + q] : 64;
+        const int ii = q < hb.degree[r] ? hb.ix[4 * r + q] : dK;
         v |= (uint32_t)ii << (8 * q);
       }
       sidx[k] = v;

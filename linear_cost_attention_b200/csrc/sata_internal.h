@@ -42,12 +42,12 @@ struct DeviceBasis {
   int64_t m = 0;
   uint32_t *idx = nullptr;
   float *w = nullptr;
-  // Tensor-core tile order (dK = 64, P == 4); null when not built.
+  // Tensor-core tile order (dK = 64 or 32, P == 4); null when not built.
   int n_tiles = 0;              // 64-feature tiles
   int64_t m_pad = 0;            // n_tiles * 64
   void *tile_desc = nullptr;      // [n_tiles] TileDesc (tile_order.h)
   int32_t *tile_row = nullptr;    // [m_pad] lexicographic row of each padded feature (-1 = pad)
-  uint32_t *slot_idx = nullptr;   // [m_pad] i | j << 8 | l << 16 of each slot (unused = 64)
+  uint32_t *slot_idx = nullptr;   // [m_pad] i | j << 8 | l << 16 of each slot (unused = dK)
   float *slot_w = nullptr;        // [m_pad] basis weight of each slot (0 = pad)
 };
 
@@ -68,7 +68,7 @@ int launch_prefill_simt(const void *q, const void *k, const void *v, float *out,
                         float *state, int B, int H, int N, int dK, int dV, int P,
                         bool bf16, bool cont, const DeviceBasis *basis, cudaStream_t stream);
 
-// Tensor-core prefill (bf16, dK = dV = 64, P = 4); basis must carry the tile order.
+// Tensor-core prefill (bf16, P = 4, dK = dV = 64 or 32); basis must carry the tile order.
 bool tc_supported(int dK, int dV, int P, bool bf16);
 // Cycles a role's wait in the tensor-core kernels may take before it gives up
 // (default: the kernels' full limit; lowered only by sata_test_set_wait_limit).

@@ -108,6 +108,8 @@ def test_workload2_fp32(P):
 def test_workload3_bf16():
     q, k, v = workload_inputs(3)
     check_prefill(q, k, v, 4, TOL["bf16"], name="workload 3 (bf16 [4,8,4096,32], P=4)")
+    # bf16 with dK = dV = 32 runs on the tensor cores
+    assert {"tc_chunk_states", "tc_readout"} <= set(launched_kernels())
 
 
 def test_workload4_bf16_sampled_heads():
@@ -146,6 +148,21 @@ def test_tensor_core_prefill_shapes(B, H, N):
     # bf16, dK = dV = 64, P = 4: the tcgen05 path
     q, k, v = make_qkv(B, H, N, 64, 64, seed=7 * N + H, dtype="bf16")
     check_prefill(q, k, v, 4, TOL["bf16"])
+    assert {"tc_chunk_states", "tc_readout"} <= set(launched_kernels())
+
+
+@pytest.mark.parametrize("B,H,N", [
+    (1, 1, 1),        # one token
+    (2, 3, 100),      # ragged, one partial key block
+    (1, 2, 4096),     # exactly one full chunk
+    (1, 1, 4224),     # one snapshot + a block of the next chunk
+    (2, 1, 9000),     # two snapshots, ragged tail
+])
+def test_tensor_core_prefill_shapes_dk32(B, H, N):
+    # bf16, dK = dV = 32, P = 4: the tcgen05 path with 4 index octets and N = 48
+    q, k, v = make_qkv(B, H, N, 32, 32, seed=11 * N + H, dtype="bf16")
+    check_prefill(q, k, v, 4, TOL["bf16"])
+    assert {"tc_chunk_states", "tc_readout"} <= set(launched_kernels())
 
 
 def test_invalid_call_raises():
@@ -213,12 +230,13 @@ def test_prefill_continue(B, H, N0, N1, dK, dV, P, dt):
     check_continue(B, H, N0, N1, dK, dV, P, dt, seed=N0 + 7 * N1)
 
 
-@pytest.mark.parametrize("N0,N1", [
-    (4224, 4300),   # prefix with one snapshot; continuation crosses a chunk boundary
-    (100, 50),      # short prefix, single-chunk continuation
+@pytest.mark.parametrize("N0,N1,d", [
+    (4224, 4300, 64),   # prefix with one snapshot; continuation crosses a chunk boundary
+    (100, 50, 64),      # short prefix, single-chunk continuation
+    (300, 4200, 32),    # dK = dV = 32
 ])
-def test_prefill_continue_tensor_core(N0, N1):
-    check_continue(1, 2, N0, N1, 64, 64, 4, "bf16", seed=N0 + N1)
+def test_prefill_continue_tensor_core(N0, N1, d):
+    check_continue(1, 2, N0, N1, d, d, 4, "bf16", seed=N0 + N1)
 
 
 @pytest.mark.parametrize("dt,dK", [("bf16", 64), ("f32", 16)])
