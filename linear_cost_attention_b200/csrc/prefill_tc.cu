@@ -10,14 +10,15 @@
 //     operand of the state MMAs and of the in-chunk P [V, 1] MMAs.  For
 //     dK = 32 it also writes Q and K padded to 64 columns with zeros, so that
 //     every tile keeps the 128-byte-swizzled layout of 64-element rows.
-//   tc_chunk_states  persistent CTAs (448 threads) over items = (head, two
+//   tc_chunk_states  persistent CTAs (448 threads) over items = (head, four
 //     128-row state tiles); the tiles S'[128 x NP] (dV+1 columns padded to
 //     the MMA's N = NP, a multiple of 16) stay in TMEM for the whole sequence.
-//     Per 128-token step: warp 0 brings the K^T and [V,1]^T boxes by TMA;
-//     warps 6-13 (one thread per basis row = TMEM lane) multiply three K^T
-//     rows for every token and store the unweighted monomials into a TMEM A
-//     stage; warp 1 (one thread) issues 16 MMAs M = 128, N = NP, K = 16 (A
-//     from TMEM, B from shared memory), the two tiles alternating.  At each
+//     Warp 0 brings 64-token K^T and [V,1]^T boxes by TMA; warps 6-13 (one
+//     TMEM lane = one lane group of four basis rows sharing two factors per
+//     thread, tile_order.h) multiply K^T rows for every token and store the
+//     unweighted monomials into a TMEM A stage of 32 tokens; warp 1 (one
+//     thread) issues 8 MMAs M = 128, N = NP, K = 16 per stage (A from TMEM, B
+//     from shared memory), the four tiles alternating on each B.  At each
 //     chunk boundary warps 2-5 copy w^2 S' into a bf16 snapshot (the state
 //     before the next chunk, "恒定计算成本的工程实现": the fixed-size state);
 //     after the last token they write w S' as the fp32 state in lexicographic
@@ -62,16 +63,17 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 }
 
 // ------------------------------------------------------------ state kernel
-constexpr int kUF = 2;          // 128-row state tiles per item
-constexpr int kUT = 128;        // tokens per step
-constexpr int kUAS = 2;         // A stages (TMEM)
-constexpr int kUKS = 4;         // K^T / V^T stages (shared memory)
-constexpr int kUGenWarps = 4 * kUF;
+constexpr int kR = kGroupRows;  // 128-row state tiles per item (rows per generator thread)
+constexpr int kAT = 32;         // tokens per A stage (two K-steps of 16)
+constexpr int kAS = 3;          // A stages in TMEM
+constexpr int kKT = 64;         // tokens per K^T / [V,1]^T stage (one TMA box of each)
+constexpr int kKS = 4;          // K^T / [V,1]^T stages in shared memory
+constexpr int kUGenWarps = 8;   // two per TMEM lane quarter, 16 tokens of each A stage each
 constexpr int kUEpiWarp0 = 2, kUGenWarp0 = 6;  // warps 2..5 epilogue, 6.. generators
 constexpr int kUThreads = 32 * (kUGenWarp0 + kUGenWarps);
 constexpr uint32_t kUTmemCols = 512;
 constexpr int kMaxDevices = 64;  // per-device launch attributes
-constexpr int kChunk = 4096;     // tokens per chunk (a multiple of the 128-token step)
+constexpr int kChunk = 4096;     // tokens per chunk (a multiple of the 128-token padding)
 
 // ------------------------------------------------------------ readout
 constexpr int kThreads = 512;
@@ -95,14 +97,15 @@ template <int DK, int DV> struct Tc {
   static constexpr float kScale = DK == 64 ? 0.125f : 0.17677669529663687f;  // 1/sqrt(dK)
   static_assert(DK == 64 || DK == 32, "the tile order exists for dK = 64 and 32");
   static_assert(NP <= (int)kRColS, "D columns below the score columns");
-  // state kernel shared memory: K^T and [V,1]^T boxes of 64 tokens, two per step
+  // state kernel shared memory: K^T and [V,1]^T boxes of 64 tokens per stage
   static constexpr uint32_t UKTh = (KR * kRow + 1023) / 1024 * 1024;
   static constexpr uint32_t UVTh = NP * kRow;
-  static constexpr uint32_t UKT = 2 * UKTh, UVT = 2 * UVTh;
-  static constexpr uint32_t UOffKT = 0, UOffVT = kUKS * UKT, UOffBar = UOffVT + kUKS * UVT;
+  static constexpr uint32_t UOffKT = 0, UOffVT = kKS * UKTh, UOffBar = UOffVT + kKS * UVTh;
   static constexpr uint32_t USmem = UOffBar + 256 + 1024;
-  static constexpr uint32_t UColA = (kUF * NP + 31) / 32 * 32;  // TMEM: D at f*NP, A from here
-  static_assert(UColA + kUAS * kUF * (kUT / 2) <= kUTmemCols, "TMEM budget");
+  // TMEM: tile f's accumulator at columns f*NP; A stages (kR tiles x 16
+  // columns of packed token pairs each) from UColA
+  static constexpr uint32_t UColA = (kR * NP + 31) / 32 * 32;
+  static_assert(UColA + kAS * kR * (kAT / 2) <= kUTmemCols, "TMEM budget");
   // readout shared memory
   static constexpr uint32_t RB = NP * kRow;    // NP x 64 snapshot tile
   static constexpr uint32_t RVT = NP * kRow;   // NP x 64-key [V,1]^T block
@@ -112,21 +115,13 @@ template <int DK, int DV> struct Tc {
   static constexpr uint32_t RSmem = ROffBar + 512 + 1024;  // barriers, TMEM slot, flag
 };
 
-// TMEM lane -> slot inside a 128-row state tile.  Within each 32-lane warp
-// quarter, lane 4c + b holds slot 8b + c: in the 8 x 8 tiles (index octets b, c)
-// a warp then reads each "c" operand row from 4 adjacent lanes and each "b"
-// operand row from every fourth lane, which shared memory serves at half the
-// cost of one row per lane & 7.
-__host__ __device__ constexpr int lane_slot(int r) {
-  return (r & ~31) | ((r & 3) << 3) | ((r >> 2) & 7);
-}
-
 struct UParams {
-  const uint32_t *slot_idx;  // [m_pad] i | j << 8 | l << 16 (dK = the ones row)
-  const float *slot_w;       // [m_pad] basis weight (0 on padding)
-  const int32_t *row_of_slot;
-  int n_mt;                  // 128-row tiles (m_pad / 128)
-  int N, C, nsnap, m, m_pad, n_batches, n_items, head0;
+  const uint64_t *grp_idx;   // [n_grp][128] j | l << 8 | i_f << (16 + 8 f) (dK = the ones row)
+  const int32_t *grp_slot;   // [n_grp][kR][128] tile-order slot (snapshot column), -1 padding
+  const int32_t *grp_row;    // [n_grp][kR][128] lexicographic basis row, -1 padding
+  const float *grp_w;        // [n_grp][kR][128] basis weight
+  int n_grp;                 // items per head
+  int N, Npad, C, nsnap, m, m_pad, n_items, head0;
   int cont;             // 1: start from the state in `state` (continued prefill)
   __nv_bfloat16 *snap;  // [G][nsnap][dV+1][m_pad]; slot 0 = initial state if cont
   float *state;         // [BH][m][dV+1]
@@ -134,15 +129,17 @@ struct UParams {
   long long wait_limit;  // cycles before a role's wait gives up (drains: full limit)
 };
 
-// One CTA per (head, kUF x 128 basis rows).  Thread = basis row = TMEM lane:
-// each generator thread forms its row's unweighted monomial x_i x_j x_l for
-// the step's tokens from the transposed keys (rows of K^T; index dK is a row of
-// ones that is zero past the sequence end) and stores them with tcgen05.st
-// straight into the A operand in TMEM (basis rows x tokens, two tokens per
-// column).  The MMA accumulates S' += m(K)^T [V, 1] with [V, 1]^T as a K-major
-// B operand (rows of V^T plus its ones row; rows dV+1.. are TMA zero fill).
-// The basis weights are applied when S' leaves TMEM: state = w S', snapshot =
-// w^2 S' (the readout then multiplies by the unweighted m(q):
+// One item = (head, kR state tiles of 128 basis rows).  Thread = TMEM lane of
+// all kR tiles: each generator thread owns the kR rows of its lane group
+// (tile_order.h), which share two factors x_j x_l and differ in the third
+// x_i; per 8 tokens it loads 2 + kR rows of K^T (index dK is a row of ones
+// that is zero past the sequence end) for kR monomials, and stores the
+// unweighted monomials with tcgen05.st straight into the A operand in TMEM
+// (basis rows x tokens, two tokens per column).  The MMA accumulates
+// S' += m(K)^T [V, 1] with [V, 1]^T as a K-major B operand (rows of V^T plus
+// its ones row; rows dV+1.. are TMA zero fill), the kR tiles' MMAs sharing
+// each B.  The basis weights are applied when S' leaves TMEM: state = w S',
+// snapshot = w^2 S' (the readout then multiplies by the unweighted m(q):
 // sum_a w_a m_a(q) w_a S'_a = phi(q) . S).
 template <int DK, int DV>
 __global__ void __launch_bounds__(kUThreads, 1)
@@ -154,24 +151,24 @@ __global__ void __launch_bounds__(kUThreads, 1)
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sKT = smem + S::UOffKT, *sVT = smem + S::UOffVT;
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S::UOffBar);
-  uint64_t *kv_full = bar, *kv_empty = bar + kUKS, *a_full = bar + 2 * kUKS,
-           *a_empty = a_full + kUAS, *snap_full = a_empty + kUAS, *snap_done = snap_full + kUF,
-           *drain = snap_done + kUF, *d_ready = drain + 1;
+  uint64_t *kv_full = bar, *kv_empty = bar + kKS, *a_full = bar + 2 * kKS,
+           *a_empty = a_full + kAS, *snap_full = a_empty + kAS, *snap_done = snap_full + kR,
+           *drain = snap_done + kR, *d_ready = drain + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(d_ready + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(d_ready + 2);
-  static_assert((2 * kUKS + 2 * kUAS + 2 * kUF + 4) * 8 <= 256, "barrier region");
+  static_assert((2 * kKS + 2 * kAS + 2 * kR + 2) * 8 + 8 <= 256, "barrier region");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kUKS; ++s) {
+    for (int s = 0; s < kKS; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], kUGenWarps);
     }
-    for (int s = 0; s < kUAS; ++s) {
+    for (int s = 0; s < kAS; ++s) {
       mbar_init(&a_full[s], kUGenWarps);
       mbar_init(&a_empty[s], 1);
     }
-    for (int f = 0; f < kUF; ++f) {
+    for (int f = 0; f < kR; ++f) {
       mbar_init(&snap_full[f], 1);
       mbar_init(&snap_done[f], 4);
     }
@@ -186,89 +183,82 @@ __global__ void __launch_bounds__(kUThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int nsub = (p.N + kUT - 1) / kUT;
-  const int sub_per_chunk = p.C / kUT;
-  auto is_event = [&](int s) {
-    return s == nsub - 1 || (((s + 1) % sub_per_chunk == 0) && (s + 1 < nsub));
+  // A stage a of an item covers tokens [32 a, 32 a + 32) and reads K/V stage
+  // a / 2; with global counters (ia over all A stages of this CTA) the K/V
+  // stage is ia / 2 because every item has an even number nA of A stages.
+  const int nA = p.Npad / kAT, nK = p.Npad / kKT;
+  const int a_per_chunk = p.C / kAT;
+  auto is_event = [&](int a) {
+    return a == nA - 1 || (((a + 1) % a_per_chunk == 0) && (a + 1 < nA));
   };
 
   if (warp == 0) {
-    // ---------------- TMA producer: K^T (dK+1 rows) and [V,1]^T (NP rows), 2 x 64 tokens
+    // ---------------- TMA producer: K^T (dK+1 rows) and [V,1]^T (NP rows), 64 tokens
     if (lane == 0) {
       prefetch_tensormap(&tmKT);
       prefetch_tensormap(&tmVT);
-      uint32_t it = 0;
+      uint32_t ik = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int hb = item / p.n_batches;
-        for (int s = 0; s < nsub; ++s, ++it) {
-          const int st = it % kUKS;
-          if (it >= kUKS && !(ok = mbar_wait(&kv_empty[st], ((it / kUKS) - 1) & 1, abort_flag,
-                                             p.err, p.wait_limit)))
+        const int hb = item / p.n_grp;
+        for (int s = 0; s < nK; ++s, ++ik) {
+          const int st = ik % kKS;
+          if (ik >= kKS && !(ok = mbar_wait(&kv_empty[st], ((ik / kKS) - 1) & 1, abort_flag,
+                                            p.err, p.wait_limit)))
             break;
-          mbar_arrive_expect_tx(&kv_full[st], 2 * S::KR * kRow + 2 * S::UVTh);
-          for (int h = 0; h < 2; ++h) {
-            tma_load_3d(sKT + st * S::UKT + h * S::UKTh, &tmKT, &kv_full[st], s * kUT + 64 * h, 0,
-                        hb);
-            tma_load_3d(sVT + st * S::UVT + h * S::UVTh, &tmVT, &kv_full[st], s * kUT + 64 * h, 0,
-                        hb);
-          }
+          mbar_arrive_expect_tx(&kv_full[st], S::KR * kRow + S::UVTh);
+          tma_load_3d(sKT + st * S::UKTh, &tmKT, &kv_full[st], s * kKT, 0, hb);
+          tma_load_3d(sVT + st * S::UVTh, &tmVT, &kv_full[st], s * kKT, 0, hb);
         }
       }
-      for (uint32_t j = it > kUKS ? it - kUKS : 0; j < it; ++j) {
+      for (uint32_t j = ik > kKS ? ik - kKS : 0; j < ik; ++j) {
         volatile int never = 0;
-        mbar_wait(&kv_full[j % kUKS], (j / kUKS) & 1, &never, p.err);
+        mbar_wait(&kv_full[j % kKS], (j / kKS) & 1, &never, p.err);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, NP, false, false);
-      uint32_t it = 0, events = 0, items = 0;
+      uint32_t ia = 0, events = 0, items = 0;
       bool after_event = false;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items) {
-        const int batch = item % p.n_batches;
-        const int nmt = min(kUF, p.n_mt - batch * kUF);
         if (p.cont) {  // the epilogue has loaded the item's initial state into TMEM
           if (!(ok = mbar_wait(d_ready, items & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
         }
-        for (int s = 0; ok && s < nsub; ++s, ++it) {
-          const int ks = it % kUKS, as = it % kUAS;
-          // a_full also covers kv_full: every generator warp waited on kv_full[ks]
-          // before arriving.  One barrier wait per step: a wait in this thread
-          // stalls until the MMAs already issued have drained.
-          if (!(ok = mbar_wait(&a_full[as], (it / kUAS) & 1, abort_flag, p.err, p.wait_limit)))
+        for (int a = 0; ok && a < nA; ++a, ++ia) {
+          const int as = ia % kAS;
+          // a_full also covers kv_full: every generator warp waited on the K/V
+          // stage before arriving.  One barrier wait per A stage: a wait in
+          // this thread stalls until the MMAs already issued have drained.
+          if (!(ok = mbar_wait(&a_full[as], (ia / kAS) & 1, abort_flag, p.err, p.wait_limit)))
             break;
           tc_fence_after();
-          const uint32_t b0 = smem_u32(sVT + ks * S::UVT);
-          const bool event = is_event(s);
           if (after_event) {
             // every tile's barrier is waited once per event, in order, so no
             // barrier can run two phases ahead of its waiter
-            for (int f = 0; ok && f < kUF; ++f)
+            for (int f = 0; ok && f < kR; ++f)
               ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err, p.wait_limit);
             if (!ok) break;
             tc_fence_after();
           }
-          // the tiles' MMAs alternate, so consecutive MMAs accumulate into
-          // different TMEM columns and do not wait for each other
+          const uint32_t b0 = smem_u32(sVT + ((ia / 2) % kKS) * S::UVTh) + (ia & 1) * 64;
+          // the kR tiles' MMAs alternate, so consecutive MMAs accumulate into
+          // different TMEM columns and share their B operand
 #pragma unroll
-          for (int k = 0; k < kUT / 16; ++k) {
-            const uint64_t bd = smem_desc_sw128(b0 + (k >> 2) * S::UVTh + 32 * (k & 3), 16, 1024);
+          for (int k = 0; k < kAT / 16; ++k) {
+            const uint64_t bd = smem_desc_sw128(b0 + 32 * k, 16, 1024);
 #pragma unroll
-            for (int f = 0; f < kUF; ++f)
-              if (f < nmt)
-                mma_bf16_ts(tmem + f * NP, tmem + S::UColA + (as * kUF + f) * (kUT / 2) + 8 * k, bd,
-                            idesc, (s > 0 || k > 0 || p.cont) ? 1u : 0u);
+            for (int f = 0; f < kR; ++f)
+              mma_bf16_ts(tmem + f * NP, tmem + S::UColA + (as * kR + f) * (kAT / 2) + 8 * k, bd,
+                          idesc, (a > 0 || k > 0 || p.cont) ? 1u : 0u);
           }
           after_event = false;
-          // one commit per step: the generators release the K^T / V^T stage
-          // once this commit has fired (each tcgen05.commit costs pipe time)
           mma_commit(&a_empty[as]);
-          if (event) {
-            for (int f = 0; f < kUF; ++f) mma_commit(&snap_full[f]);
+          if (is_event(a)) {
+            for (int f = 0; f < kR; ++f) mma_commit(&snap_full[f]);
             ++events;
             after_event = true;
           }
@@ -286,120 +276,131 @@ __global__ void __launch_bounds__(kUThreads, 1)
     uint32_t events = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int hb = item / p.n_batches, batch = item % p.n_batches;
+      const int hb = item / p.n_grp, itl = item % p.n_grp;
       if (p.cont) {
         // continued prefill: S' = S_0 / w into the TMEM tiles (the item's MMAs
         // accumulate onto it), and the snapshot before chunk 0 (slot 0) is
         // w^2 S' = w S_0.  This thread writes the same state rows at the end.
-        for (int f = 0; f < kUF; ++f) {
-          const int mt = batch * kUF + f;
-          if (mt >= p.n_mt) continue;
-          const int slot = mt * 128 + lane_slot(row);
-          const float w = p.slot_w[slot];
-          const int r = p.row_of_slot[slot];
+        for (int f = 0; f < kR; ++f) {
+          const size_t gk = ((size_t)itl * kR + f) * 128 + row;
+          const int slot = p.grp_slot[gk], r = p.grp_row[gk];
+          const float w = p.grp_w[gk];
           const float *src = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * D1;
           __nv_bfloat16 *sdst = p.snap + ((size_t)hb * p.nsnap * D1) * p.m_pad + slot;
-          uint32_t v[NP];
 #pragma unroll
-          for (int n = 0; n < NP; ++n) {
-            const float x = (n < D1 && r >= 0) ? src[n] : 0.f;
-            v[n] = __float_as_uint(w != 0.f ? x / w : 0.f);
-            if (n < D1) sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(w * x);
+          for (int j = 0; j < NP / 16; ++j) {
+            uint32_t v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int n = 16 * j + e;
+              const float x = (n < D1 && r >= 0) ? src[n] : 0.f;
+              v[e] = __float_as_uint(w != 0.f ? x / w : 0.f);
+              if (n < D1 && slot >= 0) sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(w * x);
+            }
+            tmem_st16(tmem + tl + f * NP + 16 * j, v);
           }
-#pragma unroll
-          for (int j = 0; j < NP / 16; ++j)
-            tmem_st16(tmem + tl + f * NP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(d_ready);
       }
-      for (int s = 0; ok && s < nsub; ++s) {
-        if (!is_event(s)) continue;
-        const bool boundary = s != nsub - 1;
-        const int c = boundary ? (s + 1) / sub_per_chunk - 1 + p.cont : 0;
-        for (int f = 0; ok && f < kUF; ++f) {
+      for (int a = 0; ok && a < nA; ++a) {
+        if (!is_event(a)) continue;
+        const bool boundary = a != nA - 1;
+        const int c = boundary ? (a + 1) / a_per_chunk - 1 + p.cont : 0;
+        for (int f = 0; ok && f < kR; ++f) {
           if (!(ok = mbar_wait(&snap_full[f], events & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
-          const int mt = batch * kUF + f;
-          const bool live = mt < p.n_mt;
-          const int slot = mt * 128 + lane_slot(row);
-          const float w = live ? p.slot_w[slot] : 0.f;
-          const int r = (live && !boundary) ? p.row_of_slot[slot] : -1;
+          const size_t gk = ((size_t)itl * kR + f) * 128 + row;
+          const int slot = p.grp_slot[gk];
+          const int r = boundary ? -1 : p.grp_row[gk];
+          const float w = p.grp_w[gk];
+          const float scale = boundary ? w * w : w;
           __nv_bfloat16 *sdst = p.snap + ((size_t)(hb * p.nsnap + c) * D1) * p.m_pad + slot;
           float *tdst = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * D1;
-          const float scale = boundary ? w * w : w;
-          uint32_t v[NP];
-          if (live) {
+          // 16 columns at a time: read, then store; the tile is released once
+          // every column has been read
 #pragma unroll
-            for (int j = 0; j < NP / 16; ++j)
-              tmem_ld16(tmem + tl + f * NP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+          for (int j = 0; j < NP / 16; ++j) {
+            uint32_t v[16];
+            tmem_ld16(tmem + tl + f * NP + 16 * j, v);
             tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int n = 16 * j + e;
+              if (n >= D1) continue;
+              const float x = scale * __uint_as_float(v[e]);
+              if (boundary) {
+                if (slot >= 0) sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(x);
+              } else if (r >= 0) {
+                tdst[n] = x;
+              }
+            }
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&snap_done[f]);
-          if (!live) continue;
-          if (boundary) {
-#pragma unroll
-            for (int n = 0; n < D1; ++n)
-              sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(scale * __uint_as_float(v[n]));
-          } else if (r >= 0) {
-#pragma unroll
-            for (int n = 0; n < D1; ++n) tdst[n] = scale * __uint_as_float(v[n]);
-          }
         }
         ++events;
       }
     }
   } else {
-    // ---------------- generators: one thread per basis row
-    const int g = warp - kUGenWarp0;
-    const int f = g >> 2;               // state tile of this warp
+    // ---------------- generators: one TMEM lane (lane group of kR rows) per thread
+    const int gw = warp - kUGenWarp0;
+    const int hf = gw >> 2;             // tokens [16 hf, 16 hf + 16) of every A stage
     const int q4 = warp & 3;            // TMEM lane quarter
-    const int row = 32 * q4 + lane;     // basis row inside the tile
+    const int row = 32 * q4 + lane;     // TMEM lane
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
-    constexpr uint32_t kOnes = (uint32_t)DK * 0x10101u;  // three "ones" rows
-    uint32_t it = 0;
+    uint32_t ia = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int batch = item % p.n_batches;
-      const int mt = batch * kUF + f;
-      uint32_t ix = kOnes;
-      if (mt < p.n_mt) ix = p.slot_idx[mt * 128 + lane_slot(row)];
-      const uint32_t ri = (ix & 0xff) * kRow, rj = ((ix >> 8) & 0xff) * kRow,
-                     rl = ((ix >> 16) & 0xff) * kRow;
-      const uint32_t si = (ix & 7), sj = ((ix >> 8) & 7), sl = ((ix >> 16) & 7);
-      for (int s = 0; ok && s < nsub; ++s, ++it) {
-        const int ks = it % kUKS, as = it % kUAS;
-        if (!(ok = mbar_wait(&kv_full[ks], (it / kUKS) & 1, abort_flag, p.err, p.wait_limit)))
+      const int itl = item % p.n_grp;
+      const uint64_t ix = p.grp_idx[(size_t)itl * 128 + row];
+      // byte offset of each factor row inside a K^T box, and its swizzle phase
+      const uint32_t rj = (uint32_t)(ix & 0xff), rl = (uint32_t)((ix >> 8) & 0xff);
+      uint32_t ri[kR];
+#pragma unroll
+      for (int f = 0; f < kR; ++f) ri[f] = (uint32_t)((ix >> (16 + 8 * f)) & 0xff);
+      for (int a = 0; ok && a < nA; ++a, ++ia) {
+        const int as = ia % kAS;
+        const uint32_t kv = (ia / 2) % kKS;
+        if ((ia & 1) == 0 &&
+            !(ok = mbar_wait(&kv_full[kv], ((ia / 2) / kKS) & 1, abort_flag, p.err, p.wait_limit)))
           break;
-        if (it >= kUAS) {
-          if (!(ok = mbar_wait(&a_empty[as], ((it / kUAS) - 1) & 1, abort_flag, p.err,
+        if (ia >= kAS) {
+          if (!(ok = mbar_wait(&a_empty[as], ((ia / kAS) - 1) & 1, abort_flag, p.err,
                                p.wait_limit)))
             break;
-          // the MMAs of step it - kUAS are complete and this warp read its K^T
-          // rows long ago: release that step's K^T / V^T stage
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&kv_empty[(it - kUAS) % kUKS]);
-        }
-#pragma unroll 1
-        for (int h = 0; h < kUT / 64; ++h) {  // 64 tokens (one K^T box) at a time
-          const uint32_t kt = smem_u32(sKT) + ks * S::UKT + h * S::UKTh;
-          uint32_t out[32];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 xi = lds128(kt + ri + (((uint32_t)c ^ si) << 4));
-            const uint4 xj = lds128(kt + rj + (((uint32_t)c ^ sj) << 4));
-            const uint4 xl = lds128(kt + rl + (((uint32_t)c ^ sl) << 4));
-            out[4 * c + 0] = bmul2(bmul2(xi.x, xj.x), xl.x);
-            out[4 * c + 1] = bmul2(bmul2(xi.y, xj.y), xl.y);
-            out[4 * c + 2] = bmul2(bmul2(xi.z, xj.z), xl.z);
-            out[4 * c + 3] = bmul2(bmul2(xi.w, xj.w), xl.w);
+          // the MMAs of A stage ia - kAS are complete; when that was the second
+          // A stage of its K/V stage, this warp releases the K/V stage
+          const uint32_t done = ia - kAS;
+          if (done & 1) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&kv_empty[(done / 2) % kKS]);
           }
-          tmem_st32(tmem + tl + S::UColA + (as * kUF + f) * (kUT / 2) + 32 * h, out);
         }
+        const uint32_t kt = smem_u32(sKT) + kv * S::UKTh;
+        uint32_t out[kR][8];
+#pragma unroll
+        for (int g8 = 0; g8 < 2; ++g8) {  // 8 tokens per 16-byte chunk of a K^T row
+          const uint32_t c = (ia & 1) * 4 + hf * 2 + g8;
+          const uint4 xj = lds128(kt + rj * kRow + ((c ^ (rj & 7)) << 4));
+          const uint4 xl = lds128(kt + rl * kRow + ((c ^ (rl & 7)) << 4));
+          const uint4 u = make_uint4(bmul2(xj.x, xl.x), bmul2(xj.y, xl.y), bmul2(xj.z, xl.z),
+                                     bmul2(xj.w, xl.w));
+#pragma unroll
+          for (int f = 0; f < kR; ++f) {
+            const uint4 xi = lds128(kt + ri[f] * kRow + ((c ^ (ri[f] & 7)) << 4));
+            out[f][4 * g8 + 0] = bmul2(xi.x, u.x);
+            out[f][4 * g8 + 1] = bmul2(xi.y, u.y);
+            out[f][4 * g8 + 2] = bmul2(xi.z, u.z);
+            out[f][4 * g8 + 3] = bmul2(xi.w, u.w);
+          }
+        }
+#pragma unroll
+        for (int f = 0; f < kR; ++f)
+          tmem_st8(tmem + tl + S::UColA + (as * kR + f) * (kAT / 2) + 8 * hf, out[f]);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -812,7 +813,7 @@ int launch_tc(const void *q, const void *k, const void *v, float *out, float *st
   // snapshots: the state before each chunk but the first, plus (continued
   // prefill) the initial state before chunk 0 in slot 0
   const int nsnap = (N + C - 1) / C - 1 + (cont ? 1 : 0);
-  const int Npad = ((N + kUT - 1) / kUT) * kUT;  // multiple of the 128-token step
+  const int Npad = ((N + 127) / 128) * 128;  // whole 64-token K/V stages, 128-token blocks
   const size_t snap_head = (size_t)nsnap * D1 * m_pad * 2;
   const size_t kt_head = (size_t)S::KR * Npad * 2, vt_head = (size_t)D1 * Npad * 2;
   const size_t pad_head = DK < 64 ? (size_t)Npad * 64 * 2 : 0;  // padded Q or K of one head
@@ -850,8 +851,6 @@ int launch_tc(const void *q, const void *k, const void *v, float *out, float *st
   }
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
 
-  const int n_mt = m_pad / 128;
-  const int n_batches = (n_mt + kUF - 1) / kUF;
   const int nblk = (N + 127) / 128;
   GenWeights ones;  // the readout generates unweighted monomials
   ones.w3 = ones.w3h = ones.w3s = ones.w2 = ones.w2h = ones.w1 = 1.f;
@@ -871,17 +870,18 @@ int launch_tc(const void *q, const void *k, const void *v, float *out, float *st
         reinterpret_cast<const __nv_bfloat16 *>(v), kt, vt, qpad, kpad, N, Npad, h0);
     prof_kernel_end(stream);
     UParams up;
-    up.slot_idx = basis->slot_idx;
-    up.slot_w = basis->slot_w;
-    up.row_of_slot = basis->tile_row;
-    up.n_mt = n_mt;
+    up.grp_idx = basis->grp_idx;
+    up.grp_slot = basis->grp_slot;
+    up.grp_row = basis->grp_row;
+    up.grp_w = basis->grp_w;
+    up.n_grp = basis->n_grp;
     up.N = N;
+    up.Npad = Npad;
     up.C = C;
     up.nsnap = nsnap;
     up.m = (int)basis->m;
     up.m_pad = m_pad;
-    up.n_batches = n_batches;
-    up.n_items = g * n_batches;
+    up.n_items = g * basis->n_grp;
     up.head0 = h0;
     up.cont = cont ? 1 : 0;
     up.snap = snap;

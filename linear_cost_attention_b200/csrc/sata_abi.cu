@@ -48,9 +48,10 @@ void free_basis(DeviceBasis *b) {
   cudaFree(b->idx);
   cudaFree(b->w);
   cudaFree(b->tile_desc);
-  cudaFree(b->tile_row);
-  cudaFree(b->slot_idx);
-  cudaFree(b->slot_w);
+  cudaFree(b->grp_idx);
+  cudaFree(b->grp_slot);
+  cudaFree(b->grp_row);
+  cudaFree(b->grp_w);
   delete b;
 }
 
@@ -93,33 +94,23 @@ const DeviceBasis *get_device_basis(int dK, int P, int *status) {
     }
     db->n_tiles = to.n_tiles;
     db->m_pad = (int64_t)to.n_tiles * 64;
-    // per slot: the row's index triple (unused slots point at row dK, the ones
-    // row of the transposed keys) and its weight
-    const uint32_t ones3 = (uint32_t)dK * 0x10101u;
-    std::vector<uint32_t> sidx(db->m_pad, ones3);
-    std::vector<float> sw(db->m_pad, 0.f);
-    for (int64_t k = 0; k < db->m_pad; ++k) {
-      const int32_t r = to.row_of_slot[k];
-      if (r < 0) continue;
-      uint32_t v = 0;
-      for (int q = 0; q < 3; ++q) {
-        const int ii = q < hb.degree[r] ? hb.ix[4 * r + q] : dK;
-        v |= (uint32_t)ii << (8 * q);
-      }
-      sidx[k] = v;
-      sw[k] = (float)hb.weight[r];
+    // row groups of the state kernel (their slots index the padded tile order)
+    StateGroups sg;
+    if (!build_state_groups(dK, to, &sg)) {
+      free_basis(db);
+      *status = SATA_ERR_CUDA;
+      return nullptr;
     }
-    ok = cudaMalloc(&db->slot_idx, sidx.size() * sizeof(uint32_t)) == cudaSuccess &&
-         cudaMalloc(&db->slot_w, sw.size() * sizeof(float)) == cudaSuccess &&
-         cudaMemcpy(db->slot_idx, sidx.data(), sidx.size() * sizeof(uint32_t),
-                    cudaMemcpyHostToDevice) == cudaSuccess &&
-         cudaMemcpy(db->slot_w, sw.data(), sw.size() * sizeof(float), cudaMemcpyHostToDevice) ==
-             cudaSuccess &&
+    db->n_grp = sg.n_items;
+    auto upload = [&](auto **dst, const auto &vec) {
+      const size_t bytes = vec.size() * sizeof(vec[0]);
+      return cudaMalloc((void **)dst, bytes) == cudaSuccess &&
+             cudaMemcpy(*dst, vec.data(), bytes, cudaMemcpyHostToDevice) == cudaSuccess;
+    };
+    ok = upload(&db->grp_idx, sg.lane_idx) && upload(&db->grp_slot, sg.slot) &&
+         upload(&db->grp_row, sg.row) && upload(&db->grp_w, sg.weight) &&
          cudaMalloc(&db->tile_desc, to.tiles.size() * sizeof(TileDesc)) == cudaSuccess &&
-         cudaMalloc(&db->tile_row, to.row_of_slot.size() * sizeof(int32_t)) == cudaSuccess &&
          cudaMemcpy(db->tile_desc, to.tiles.data(), to.tiles.size() * sizeof(TileDesc),
-                    cudaMemcpyHostToDevice) == cudaSuccess &&
-         cudaMemcpy(db->tile_row, to.row_of_slot.data(), to.row_of_slot.size() * sizeof(int32_t),
                     cudaMemcpyHostToDevice) == cudaSuccess;
   }
   // cudaMemcpy from pageable memory may return before the DMA has landed, and

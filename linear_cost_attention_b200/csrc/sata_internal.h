@@ -42,13 +42,15 @@ struct DeviceBasis {
   int64_t m = 0;
   uint32_t *idx = nullptr;
   float *w = nullptr;
-  // Tensor-core tile order (dK = 64 or 32, P == 4); null when not built.
-  int n_tiles = 0;              // 64-feature tiles
+  // Tensor-core tables (dK = 64 or 32, P == 4); null when not built.
+  int n_tiles = 0;              // 64-feature tiles of the tile order (readout, snapshots)
   int64_t m_pad = 0;            // n_tiles * 64
-  void *tile_desc = nullptr;      // [n_tiles] TileDesc (tile_order.h)
-  int32_t *tile_row = nullptr;    // [m_pad] lexicographic row of each padded feature (-1 = pad)
-  uint32_t *slot_idx = nullptr;   // [m_pad] i | j << 8 | l << 16 of each slot (unused = dK)
-  float *slot_w = nullptr;        // [m_pad] basis weight of each slot (0 = pad)
+  void *tile_desc = nullptr;    // [n_tiles] TileDesc (tile_order.h)
+  int n_grp = 0;                // state-kernel items per head (StateGroups, tile_order.h)
+  uint64_t *grp_idx = nullptr;  // [n_grp][128] shared and third factor rows of each lane group
+  int32_t *grp_slot = nullptr;  // [n_grp][4][128] tile-order slot of each row (-1 = pad)
+  int32_t *grp_row = nullptr;   // [n_grp][4][128] lexicographic row (-1 = pad)
+  float *grp_w = nullptr;       // [n_grp][4][128] basis weight (0 = pad)
 };
 
 // Returns the cached tables for the current device (builds them on first use).

@@ -135,4 +135,120 @@ bool build_tile_order(int dK, TileOrder *out) {
   return true;
 }
 
+bool build_state_groups(int dK, const TileOrder &to, StateGroups *out) {
+  if ((dK != 64 && dK != 32) || to.dK != dK) return false;
+  const int G = dK / 8;
+  const int ONES = dK, PAD = -1;
+  HostBasis hb = build_host_basis(dK, 4);
+  std::map<uint32_t, int32_t> lex;
+  for (int64_t r = 0; r < hb.m; ++r) {
+    const int deg = hb.degree[r];
+    int ix[3] = {-1, -1, -1};
+    for (int s = 0; s < deg; ++s) ix[s] = hb.ix[4 * r + s];
+    lex[tuple_key(deg, ix[0], ix[1], ix[2])] = (int32_t)r;
+  }
+  std::vector<int32_t> slot_of_row(hb.m, -1);
+  for (size_t k = 0; k < to.row_of_slot.size(); ++k)
+    if (to.row_of_slot[k] >= 0) slot_of_row[to.row_of_slot[k]] = (int32_t)k;
+
+  struct LaneGroup {
+    int j, l, third[kGroupRows];
+  };
+  std::vector<LaneGroup> lg;
+  auto add = [&](int j, int l, int t0, int t1, int t2, int t3) {
+    lg.push_back({j, l, {t0, t1, t2, t3}});
+  };
+  // degree 3, three distinct octets gi < gj < gl: third factor 8 gi + 4 ahi + f
+  // (uniform in each warp), shared x_j x_l over the octets gj, gl
+  for (int gi = 0; gi < G; ++gi)
+    for (int gj = gi + 1; gj < G; ++gj)
+      for (int gl = gj + 1; gl < G; ++gl)
+        for (int ahi = 0; ahi < 2; ++ahi)
+          for (int bh = 0; bh < 2; ++bh)
+            for (int lane = 0; lane < 32; ++lane) {
+              const int b = 4 * bh + (lane & 3), c = lane >> 2;
+              const int t = 8 * gi + 4 * ahi;
+              add(8 * gj + b, 8 * gl + c, t, t + 1, t + 2, t + 3);
+            }
+  // degree 3 with a pair a <= b inside octet g and the third index in octet
+  // g' != g: shared pair, third factor 8 g' + 4 h + f (uniform per (g', h))
+  for (int g2 = 0; g2 < G; ++g2)
+    for (int h = 0; h < 2; ++h)
+      for (int g = 0; g < G; ++g) {
+        if (g == g2) continue;
+        for (int a = 0; a < 8; ++a)
+          for (int b = a; b < 8; ++b) {
+            const int t = 8 * g2 + 4 * h;
+            add(8 * g + a, 8 * g + b, t, t + 1, t + 2, t + 3);
+          }
+      }
+  // degree 3 inside one octet: shared pair a <= b, third c = b..7
+  for (int g = 0; g < G; ++g)
+    for (int a = 0; a < 8; ++a)
+      for (int b = a; b < 8; ++b)
+        for (int c0 = b; c0 < 8; c0 += kGroupRows) {
+          int t[kGroupRows];
+          for (int f = 0; f < kGroupRows; ++f) t[f] = c0 + f < 8 ? 8 * g + c0 + f : PAD;
+          add(8 * g + a, 8 * g + b, t[0], t[1], t[2], t[3]);
+        }
+  // degree 2 (u <= w): shared x_w and ones, third factor u
+  for (int w = 0; w < dK; ++w)
+    for (int u0 = 0; u0 <= w; u0 += kGroupRows) {
+      int t[kGroupRows];
+      for (int f = 0; f < kGroupRows; ++f) t[f] = u0 + f <= w ? u0 + f : PAD;
+      add(w, ONES, t[0], t[1], t[2], t[3]);
+    }
+  // degree 1 and degree 0
+  for (int u0 = 0; u0 < dK; u0 += kGroupRows) add(ONES, ONES, u0, u0 + 1, u0 + 2, u0 + 3);
+  add(ONES, ONES, ONES, PAD, PAD, PAD);
+  while (lg.size() % 128) add(ONES, ONES, PAD, PAD, PAD, PAD);
+
+  const int n_items = (int)(lg.size() / 128);
+  out->n_items = n_items;
+  // tile-order slots that hold no row: given to padding rows (weight 0), so
+  // that every snapshot column is written (with zeros there)
+  std::vector<int32_t> free_slots;
+  for (size_t k = 0; k < to.row_of_slot.size(); ++k)
+    if (to.row_of_slot[k] < 0) free_slots.push_back((int32_t)k);
+  out->lane_idx.assign((size_t)n_items * 128, 0);
+  out->slot.assign((size_t)n_items * kGroupRows * 128, -1);
+  out->row.assign((size_t)n_items * kGroupRows * 128, -1);
+  out->weight.assign((size_t)n_items * kGroupRows * 128, 0.f);
+  std::vector<int> hits(hb.m, 0);
+  for (int it = 0; it < n_items; ++it)
+    for (int lane = 0; lane < 128; ++lane) {
+      const LaneGroup &q = lg[(size_t)it * 128 + lane];
+      uint64_t packed = (uint64_t)q.j | (uint64_t)q.l << 8;
+      for (int f = 0; f < kGroupRows; ++f) {
+        const int t = q.third[f];
+        packed |= (uint64_t)(t == PAD ? ONES : t) << (16 + 8 * f);
+        if (t == PAD) {
+          if (!free_slots.empty()) {
+            out->slot[((size_t)it * kGroupRows + f) * 128 + lane] = free_slots.back();
+            free_slots.pop_back();
+          }
+          continue;
+        }
+        int v[3] = {t, q.j, q.l}, idx[3], deg = 0;
+        for (int s2 = 0; s2 < 3; ++s2)
+          if (v[s2] != ONES) idx[deg++] = v[s2];
+        std::sort(idx, idx + deg);
+        auto itr = lex.find(tuple_key(deg, deg > 0 ? idx[0] : -1, deg > 1 ? idx[1] : -1,
+                                      deg > 2 ? idx[2] : -1));
+        if (itr == lex.end()) return false;
+        const int32_t r = itr->second;
+        const size_t k = ((size_t)it * kGroupRows + f) * 128 + lane;
+        out->slot[k] = slot_of_row[r];
+        out->row[k] = r;
+        out->weight[k] = (float)hb.weight[r];
+        if (slot_of_row[r] < 0) return false;
+        hits[r]++;
+      }
+      out->lane_idx[(size_t)it * 128 + lane] = packed;
+    }
+  for (int64_t r = 0; r < hb.m; ++r)
+    if (hits[r] != 1) return false;
+  return free_slots.empty();  // every slot of the tile order is written
+}
+
 }  // namespace sata

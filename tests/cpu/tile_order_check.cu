@@ -4,10 +4,13 @@
 //   1. every basis row appears in exactly one tile slot;
 //   2. for random bf16 rows, every generated feature equals the basis weight
 //      times the product of its indexed entries, up to bf16 rounding;
+//   3. the state kernel's row groups hold every basis row and every tile-order
+//      slot once, and each row's shared and third factors are its indices;
 // for dK = 64 (8 index octets) and dK = 32 (4 octets).
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <random>
 #include <vector>
 
@@ -91,8 +94,57 @@ int check(int dK, int want_tiles) {
   return bad ? 1 : 0;
 }
 
+// The state kernel's row groups: each row's factors (j, l, i_f, with dK
+// standing for a ones row) are its index tuple; every basis row and every slot
+// of the tile order (padded to an even tile count, as the library does) is
+// used exactly once, with the row's weight.
+int check_groups(int dK) {
+  TileOrder to;
+  if (!build_tile_order(dK, &to)) return 1;
+  if (to.n_tiles % 2) {
+    to.tiles.push_back({T_PAD, 0, 0, 0, 0, 0, 0, 0});
+    to.row_of_slot.insert(to.row_of_slot.end(), 64, -1);
+    to.n_tiles++;
+  }
+  StateGroups sg;
+  if (!build_state_groups(dK, to, &sg)) {
+    printf("FAIL build_state_groups dK=%d\n", dK);
+    return 1;
+  }
+  HostBasis hb = build_host_basis(dK, 4);
+  std::vector<int> row_hits(hb.m, 0), slot_hits(to.row_of_slot.size(), 0);
+  long bad = 0;
+  for (int it = 0; it < sg.n_items; ++it)
+    for (int lane = 0; lane < 128; ++lane) {
+      const uint64_t ix = sg.lane_idx[(size_t)it * 128 + lane];
+      for (int f = 0; f < kGroupRows; ++f) {
+        const size_t k = ((size_t)it * kGroupRows + f) * 128 + lane;
+        const int r = sg.row[k], slot = sg.slot[k];
+        if (slot >= 0) slot_hits[slot]++;
+        if (r < 0) {
+          if (sg.weight[k] != 0.f || (slot >= 0 && to.row_of_slot[slot] >= 0)) ++bad;
+          continue;
+        }
+        row_hits[r]++;
+        int fac[3] = {(int)((ix >> (16 + 8 * f)) & 0xff), (int)(ix & 0xff), (int)((ix >> 8) & 0xff)};
+        std::vector<int> got, want;
+        for (int q = 0; q < 3; ++q)
+          if (fac[q] != dK) got.push_back(fac[q]);
+        for (int q = 0; q < hb.degree[r]; ++q) want.push_back(hb.ix[4 * r + q]);
+        std::sort(got.begin(), got.end());
+        if (got != want || slot < 0 || to.row_of_slot[slot] != r ||
+            sg.weight[k] != (float)hb.weight[r])
+          ++bad;
+      }
+    }
+  for (int64_t r = 0; r < hb.m; ++r) bad += row_hits[r] != 1;
+  for (size_t k = 0; k < slot_hits.size(); ++k) bad += slot_hits[k] != 1;
+  printf("dK %d: %d state items, bad %ld\n", dK, sg.n_items, bad);
+  return bad ? 1 : 0;
+}
+
 int main() {
-  int fails = check<8>(64, 749) + check<4>(32, 103);
+  int fails = check<8>(64, 749) + check<4>(32, 103) + check_groups(64) + check_groups(32);
   if (fails) {
     printf("FAIL\n");
     return 1;
