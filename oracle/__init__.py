@@ -20,6 +20,9 @@ Sources (web pages; cited by title and section):
 * [Attn-var] "Transformer 注意力机制变体与长序列建模优化：从 O(n²) 到线性注意力的工程演进"
   (mokono.cn), section "2.1 标准注意力实现与瓶颈分析": layout
   (batch, heads, seq_len, dim) and score scale dim**-0.5.
+* [SATA-faq] "对称感知泰勒近似实现恒定Token成本注意力机制" (ai-stack.site),
+  FAQ 5 (models trained from scratch with the method: the reason for a
+  backward pass).
 
 Readings where the pages are silent:
 degrees 0..P-1; inclusive causal mask j <= i; one normaliser shared by all
@@ -36,6 +39,7 @@ from .sata import (
     taylor_kernel,
     feature_map,
     quadratic_form,
+    attention_grad,
     conditioning,
     feature_form,
     decode_step,
@@ -47,7 +51,8 @@ from .sata import (
 
 __all__ = [
     "basis_rows", "basis_weights", "basis_all", "multiplicity_factorial",
-    "taylor_kernel", "feature_map", "quadratic_form", "conditioning", "feature_form",
+    "taylor_kernel", "feature_map", "quadratic_form", "attention_grad", "conditioning",
+    "feature_form",
     "decode_step", "final_state", "softmax_attention", "basis_total",
     "flops_per_token_counted",
 ]

@@ -13,6 +13,8 @@ Definition followed (per head; s_ij = q_i.k_j / sqrt(d_K), the dim**-0.5 scale o
 definition unchanged; so the quadratic form above and the feature-map form
 (per-token update of a fixed-size state, section "恒定计算成本的工程实现") must
 agree up to rounding.  All arithmetic is float64 from the exact input values.
+[SATA-faq] is "对称感知泰勒近似实现恒定Token成本注意力机制" (ai-stack.site), whose
+FAQ 5 reports models trained from scratch with the method (attention_grad).
 """
 from __future__ import annotations
 
@@ -93,6 +95,46 @@ def quadratic_form(q, k, v, P: int, row_block: int = 1024):
                 num[b, h, i0:i1] = t @ v[b, h, :i1]
                 den[b, h, i0:i1] = t.sum(axis=1)
     return num, den, num / den[..., None]
+
+
+def attention_grad(q, k, v, dout, P: int):
+    """Gradients of L = sum(dout * out) with respect to q, k, v, where out is
+    the definition above: the backward pass a training step needs ([SATA-faq],
+    FAQ 5, on training models with the method from scratch).  Chain rule through the
+    definition, per head, with T = T_P(s) and s = q k^T / sqrt(d_K) on j <= i:
+
+        dnum_i = dout_i / den_i
+        dden_i = -(dout_i . out_i) / den_i
+        dT_ij  = dnum_i . v_j + dden_i
+        dv_j   = sum_{i >= j} T_ij dnum_i
+        ds_ij  = dT_ij * T_{P-1}(s_ij)        (d/ds of sum_{p<P} s^p/p!)
+        dq_i   = sum_{j <= i} ds_ij k_j / sqrt(d_K)
+        dk_j   = sum_{i >= j} ds_ij q_i / sqrt(d_K)
+
+    Returns (dq, dk, dv) with the shapes of q, k, v.  O(N^2) per head.
+    """
+    q, k, v = _heads(q, k, v)
+    dout = _f64(dout)
+    B, H, N, dK = q.shape
+    scale = 1.0 / math.sqrt(dK)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    mask = np.arange(N)[None, :] <= np.arange(N)[:, None]
+    for b in range(B):
+        for h in range(H):
+            s = (q[b, h] @ k[b, h].T) * scale
+            T = np.where(mask, taylor_kernel(s, P), 0.0)
+            Td = np.where(mask, taylor_kernel(s, P - 1), 0.0)
+            num = T @ v[b, h]
+            den = T.sum(axis=1)
+            out = num / den[:, None]
+            dnum = dout[b, h] / den[:, None]
+            dden = -(dout[b, h] * out).sum(axis=1) / den
+            dT = np.where(mask, dnum @ v[b, h].T + dden[:, None], 0.0)
+            dv[b, h] = T.T @ dnum
+            ds = dT * Td
+            dq[b, h] = (ds @ k[b, h]) * scale
+            dk[b, h] = (ds.T @ q[b, h]) * scale
+    return dq, dk, dv
 
 
 def conditioning(q, k, P: int, row_block: int = 1024) -> np.ndarray:

@@ -371,3 +371,63 @@ def test_pins_catch_planted_mistakes():
     bn, bd = brute.brute_attention(qq[0, 0], kk[0, 0], vv[0, 0], 3)
     sn, sd, _ = oracle.quadratic_form(kk, qq, vv, 3)
     assert _rowerr(sn[0, 0], sd[0, 0], bn, bd) > 1e-6
+
+
+# ---------------------------------------------------------------- backward pass
+
+def _loss(q, k, v, dout, P):
+    return float((oracle.quadratic_form(q, k, v, P)[2] * dout).sum())
+
+
+@pytest.mark.parametrize("P", [2, 3, 4, 5])
+def test_gradient_matches_finite_differences(P):
+    # central differences of the definition itself (a computation independent
+    # of the chain rule in attention_grad), element by element
+    r = _rng(40 + P)
+    B, H, N, dK, dV = 1, 2, 6, 3, 2
+    q, k, v = (r.standard_normal((B, H, N, d)) for d in (dK, dK, dV))
+    dout = r.standard_normal((B, H, N, dV))
+    dq, dk, dv = oracle.attention_grad(q, k, v, dout, P)
+    eps = 1e-6
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            old = x[idx]
+            x[idx] = old + eps
+            lp = _loss(q, k, v, dout, P)
+            x[idx] = old - eps
+            lm = _loss(q, k, v, dout, P)
+            x[idx] = old
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert np.max(np.abs(fd - g)) <= 1e-6 * max(1.0, np.max(np.abs(g))), np.max(np.abs(fd - g))
+
+
+def test_gradient_P1_closed_form():
+    # P = 1: out_i = mean(v_0..v_i) does not depend on q, k, and
+    # dv_j = sum_{i >= j} dout_i / (i + 1)
+    r = _rng(77)
+    q, k, v = (r.standard_normal((1, 1, 7, 4)) for _ in range(3))
+    dout = r.standard_normal((1, 1, 7, 4))
+    dq, dk, dv = oracle.attention_grad(q, k, v, dout, 1)
+    assert np.all(dq == 0) and np.all(dk == 0)
+    want = np.array([sum(dout[0, 0, i] / (i + 1) for i in range(j, 7)) for j in range(7)])
+    assert np.allclose(dv[0, 0], want, rtol=1e-14, atol=1e-14)
+
+
+def test_gradient_catches_a_dropped_normaliser_term():
+    # planted mistake, in a copy on the CPU: leave out d(den) and the finite
+    # differences of the definition disagree
+    r = _rng(5)
+    q, k, v = (r.standard_normal((1, 1, 5, 3)) for _ in range(3))
+    dout = r.standard_normal((1, 1, 5, 3))
+    P = 4
+    s = (q[0, 0] @ k[0, 0].T) / math.sqrt(3)
+    mask = np.tril(np.ones((5, 5), dtype=bool))
+    T = np.where(mask, oracle.taylor_kernel(s, P), 0.0)
+    den = T.sum(1)
+    wrong_dv = T.T @ (dout[0, 0] / den[:, None])  # dv is right without the den term
+    wrong_dq = ((np.where(mask, (dout[0, 0] / den[:, None]) @ v[0, 0].T, 0.0)
+                 * np.where(mask, oracle.taylor_kernel(s, P - 1), 0.0)) @ k[0, 0]) / math.sqrt(3)
+    dq, _, dv = oracle.attention_grad(q, k, v, dout, P)
+    assert np.allclose(dv[0, 0], wrong_dv, rtol=1e-12)
+    assert not np.allclose(dq[0, 0], wrong_dq, rtol=1e-3)
