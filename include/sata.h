@@ -130,6 +130,27 @@ int sata_decode_step(const void *q, const void *k, const void *v, float *state,
                      float *out, int B, int H, int dK, int dV, int P,
                      sata_dtype dt, sata_stream_t stream);
 
+/* Backward pass: the gradients of L = sum(dout * out) with respect to q, k
+ * and v, where out is sata_prefill's output for the same q, k, v, P
+ * ("对称感知泰勒近似实现恒定Token成本注意力机制", FAQ 5: models are trained from
+ * scratch with the method).  With T_ij = T_P(s_ij) on j <= i,
+ *   dnum_i = dout_i / den_i, dden_i = -(dout_i . out_i) / den_i,
+ *   ds_ij = (dnum_i . v_j + dden_i) T_{P-1}(s_ij),
+ *   dq_i = sum_{j<=i} ds_ij k_j / sqrt(dK), dk_j = sum_{i>=j} ds_ij q_i / sqrt(dK),
+ *   dv_j = sum_{i>=j} T_ij dnum_i,
+ * evaluated over (query, key) tiles in fp32 on CUDA cores: exact up to
+ * rounding, with a cost quadratic in N (the forward's constant-cost state is
+ * not used).  q, k [B,H,N,dK] and v [B,H,N,dV] in dtype dt; dout
+ * [B,H,N,dV], dq, dk [B,H,N,dK] and dv [B,H,N,dV] float; outputs must not
+ * overlap each other or the inputs.  Supports every (dK, dV, P) of
+ * sata_prefill.  Uses the library workspace (B*H*N*(dV+1) floats).
+ * Returns SATA_OK, SATA_ERR_INVALID_ARG, SATA_ERR_UNSUPPORTED, SATA_ERR_NOMEM
+ * or SATA_ERR_CUDA. */
+int sata_attention_backward(const void *q, const void *k, const void *v,
+                            const float *dout, float *dq, float *dk, float *dv,
+                            int B, int H, int N, int dK, int dV, int P,
+                            sata_dtype dt, sata_stream_t stream);
+
 /* ---- Mixed-precision decode state ("硬件优化路径与当前局限": fp16 storage
  * halves the state's bandwidth).  The state of every head is stored as two
  * arrays: its first m_lo rows (every row of degree <= 2, m_lo =

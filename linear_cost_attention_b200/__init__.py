@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.sata_state_join.restype = i
     L.sata_decode_step_mixed.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     L.sata_decode_step_mixed.restype = i
+    L.sata_attention_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    L.sata_attention_backward.restype = i
     L.sata_test_set_wait_limit.argtypes = [ctypes.c_longlong]
     L.sata_test_set_wait_limit.restype = ctypes.c_longlong
     _lib = L
@@ -190,6 +192,15 @@ def sata_decode_step_mixed(q, k, v, state_lo, state_hi, out, B, H, dK, dV, P, dt
         raise SataError(st, "sata_decode_step_mixed")
 
 
+def sata_attention_backward(q, k, v, dout, dq, dk, dv, B, H, N, dK, dV, P, dtype,
+                            stream=None) -> None:
+    st = lib().sata_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                                       _ptr(dv), B, H, N, dK, dV, P, _dtype_code(dtype),
+                                       _stream(stream))
+    if st != SATA_OK:
+        raise SataError(st, "sata_attention_backward")
+
+
 def sata_get_error(stream=None) -> int:
     return int(lib().sata_get_error(_stream(stream)))
 
@@ -268,6 +279,21 @@ def prefill_continue(q, k, v, state, P: int, out=None, stream=None):
         out = torch.empty(B, H, N, dV, device=q.device, dtype=torch.float32)
     sata_prefill_continue(q, k, v, out, state, B, H, N, dK, dV, P, q.dtype, stream)
     return out
+
+
+def attention_backward(q, k, v, dout, P: int, stream=None):
+    """Gradients (dq, dk, dv), fp32, of sum(dout * out) for out = prefill(q, k, v, P)[0]."""
+    import torch
+
+    _check_qkv(q, k, v)
+    B, H, N, dK = q.shape
+    dV = v.shape[-1]
+    dout = dout.contiguous().float()
+    dq = torch.empty(B, H, N, dK, device=q.device, dtype=torch.float32)
+    dk = torch.empty_like(dq)
+    dv = torch.empty(B, H, N, dV, device=q.device, dtype=torch.float32)
+    sata_attention_backward(q, k, v, dout, dq, dk, dv, B, H, N, dK, dV, P, q.dtype, stream)
+    return dq, dk, dv
 
 
 def decode_step(q, k, v, state, P: int, out=None, stream=None):

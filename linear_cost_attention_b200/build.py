@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsata.so")
 
 SOURCES = ["sata_abi.cu", "basis.cpp", "tile_order.cu", "prefill_simt.cu", "prefill_tc.cu",
-           "decode.cu", "decode_noalloc.cu", "decode_bulk.cu"]
+           "decode.cu", "decode_noalloc.cu", "decode_bulk.cu", "backward.cu"]
 HEADERS = ["sata_internal.h", "common.cuh", "tc_common.cuh", "tile_gen.cuh", "tile_order.h"]
 
 NVCC_FLAGS = [

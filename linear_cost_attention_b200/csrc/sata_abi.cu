@@ -259,6 +259,8 @@ extern "C" const char *sata_kernel_name(int id) {
     case K_TC_READOUT: return "tc_readout";
     case K_TC_PREP: return "tc_prep";
     case K_DECODE_BULK: return "decode_bulk";
+    case K_BWD_ROWS: return "bwd_rows";
+    case K_BWD_COLS: return "bwd_cols";
   }
   return "unknown";
 }
@@ -443,6 +445,37 @@ extern "C" int sata_decode_step_mixed(const void *q, const void *k, const void *
   return launch_decode_bulk(q, k, v, state_lo, m > m_lo ? state_hi : nullptr, B, H, dK, dV,
                             (int)m_lo, (int)(m - m_lo), dt == SATA_BF16, basis, out,
                             (cudaStream_t)stream);
+}
+
+extern "C" int sata_attention_backward(const void *q, const void *k, const void *v,
+                                       const float *dout, float *dq, float *dk, float *dv, int B,
+                                       int H, int N, int dK, int dV, int P, sata_dtype dt,
+                                       sata_stream_t stream) {
+  if (!q || !k || !v || !dout || !dq || !dk || !dv) return SATA_ERR_INVALID_ARG;
+  const void *ptrs[7] = {q, k, v, dout, dq, dk, dv};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return SATA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return SATA_ERR_INVALID_ARG;
+  if (dt != SATA_F32 && dt != SATA_BF16) return SATA_ERR_INVALID_ARG;
+  if (!supported_dim(dK) || !supported_dim(dV) || P < 1 || P > kMaxP) return SATA_ERR_UNSUPPORTED;
+  const long long BHN = (long long)B * H * N;
+  if (BHN * (dK > dV + 1 ? dK : dV + 1) >= (1LL << 31)) return SATA_ERR_INVALID_ARG;
+  const size_t es = dt == SATA_F32 ? 4 : 2;
+  const size_t nq = BHN * dK * es, nv = BHN * dV * es, ndq = BHN * dK * 4, ndv = BHN * dV * 4;
+  const void *ins[4] = {q, k, v, dout};
+  const size_t nin[4] = {nq, nq, nv, ndv};
+  const void *outs[3] = {dq, dk, dv};
+  const size_t nout[3] = {ndq, ndq, ndv};
+  for (int o = 0; o < 3; ++o) {
+    for (int i = 0; i < 4; ++i)
+      if (overlaps(outs[o], nout[o], ins[i], nin[i])) return SATA_ERR_INVALID_ARG;
+    for (int o2 = o + 1; o2 < 3; ++o2)
+      if (overlaps(outs[o], nout[o], outs[o2], nout[o2])) return SATA_ERR_INVALID_ARG;
+  }
+  std::lock_guard<std::recursive_mutex> lock(g_mutex);  // one call at a time
+  prof_call_begin();
+  return launch_backward(q, k, v, dout, dq, dk, dv, B, H, N, dK, dV, P, dt == SATA_BF16,
+                         (cudaStream_t)stream);
 }
 
 extern "C" int sata_get_error(sata_stream_t stream) {

@@ -94,6 +94,11 @@ int launch_decode_bulk(const void *q, const void *k, const void *v, float *lo, v
 int launch_state_convert(bool split, float *state, float *lo, void *hi, long long BH, int m,
                          int m_lo, int D1, cudaStream_t stream);
 
+// Gradients of sum(dout * out) w.r.t. q, k, v (fp32 outputs, CUDA cores).
+int launch_backward(const void *q, const void *k, const void *v, const float *dout, float *dq,
+                    float *dk, float *dv, int B, int H, int N, int dK, int dV, int P, bool bf16,
+                    cudaStream_t stream);
+
 // Decode with caller-supplied basis tables (packed as in DeviceBasis) and
 // partial-sum scratch y of at least B*H*(dV+1) floats.
 int launch_decode_scratch(const void *q, const void *k, const void *v, float *state, float *out,
@@ -110,6 +115,8 @@ enum KernelId {
   K_TC_READOUT = 6,
   K_TC_PREP = 7,
   K_DECODE_BULK = 8,
+  K_BWD_ROWS = 9,
+  K_BWD_COLS = 10,
 };
 void prof_call_begin();                          // start of an entry-point call
 void prof_kernel_begin(cudaStream_t s, int id);  // before a launch

@@ -171,3 +171,17 @@ def test_mixed_state_calls_rejected_on_host():
         sata.SATA_ERR_INVALID_ARG                                 # missing fp16 array
     assert dm(A, 2 * A, 3 * A, 4 * A, 5 * A, A, 1, 1, 8, 32, 4, 1, None) == \
         sata.SATA_ERR_INVALID_ARG                                 # out aliases q
+
+
+def test_backward_call_rejected_on_host():
+    L = sata.lib()
+    A = 1 << 20
+    bw = L.sata_attention_backward
+    args = (1, 1, 8, 8, 8, 4, 0, None)
+    # every call below must fail validation: nothing may reach a launch
+    assert bw(None, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 7 * A, *args) == sata.SATA_ERR_INVALID_ARG
+    assert bw(A, 2 * A, 3 * A, 4 * A, 5 * A + 4, 6 * A, 7 * A, *args) == sata.SATA_ERR_INVALID_ARG
+    assert bw(A, 2 * A, 3 * A, 4 * A, A, 6 * A, 7 * A, *args) == sata.SATA_ERR_INVALID_ARG  # dq = q
+    assert bw(A, 2 * A, 3 * A, 4 * A, 5 * A, 5 * A, 7 * A, *args) == sata.SATA_ERR_INVALID_ARG
+    assert bw(A, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 7 * A, 1, 1, 8, 12, 8, 4, 0, None) == \
+        sata.SATA_ERR_UNSUPPORTED
