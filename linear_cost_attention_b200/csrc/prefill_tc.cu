@@ -78,15 +78,13 @@ constexpr int kChunk = 4096;     // tokens per chunk (a multiple of the 128-toke
 // ------------------------------------------------------------ readout
 constexpr int kThreads = 512;
 constexpr int kMaxTiles = 768;           // tile table capacity in smem
-constexpr int kRTS = 4;                  // feature tiles per pipeline stage
-constexpr int kRStages = 2;              // phi(Q) stages, in TMEM (32 columns per tile)
-constexpr int kRBS = 3;                  // snapshot stages (kRTS tiles each)
+constexpr int kRTS = 2;                  // feature tiles per pipeline stage
+constexpr int kRStages = 2;              // phi(Q) stages, in TMEM (2 blocks x 32 columns per tile)
+constexpr int kRBS = 4;                  // snapshot stages (kRTS tiles each)
 constexpr int kKB = 64;                  // keys per in-chunk block
 constexpr uint32_t kRTile = 128 * kRow;  // 128 tokens x 64 features: 16 KiB
 constexpr uint32_t kRKB = kKB * kRow;    // 64 keys x 64 dims: 8 KiB
-constexpr uint32_t kRColS = 96, kRColA = 160;  // TMEM: D 0..NP-1, scores 96..159, A stages
 constexpr uint32_t kRTmemCols = 512;
-static_assert(kRColA + 32 * kRTS * kRStages <= kRTmemCols, "TMEM budget");
 
 // Shapes of one (dK, dV) instantiation.
 template <int DK, int DV> struct Tc {
@@ -96,7 +94,7 @@ template <int DK, int DV> struct Tc {
   static constexpr int G = DK / 8;                 // index octets of the tile order
   static constexpr float kScale = DK == 64 ? 0.125f : 0.17677669529663687f;  // 1/sqrt(dK)
   static_assert(DK == 64 || DK == 32, "the tile order exists for dK = 64 and 32");
-  static_assert(NP <= (int)kRColS, "D columns below the score columns");
+
   // state kernel shared memory: K^T and [V,1]^T boxes of 64 tokens per stage
   static constexpr uint32_t UKTh = (KR * kRow + 1023) / 1024 * 1024;
   static constexpr uint32_t UVTh = NP * kRow;
@@ -106,10 +104,14 @@ template <int DK, int DV> struct Tc {
   // columns of packed token pairs each) from UColA
   static constexpr uint32_t UColA = (kR * NP + 31) / 32 * 32;
   static_assert(UColA + kAS * kR * (kAT / 2) <= kUTmemCols, "TMEM budget");
+  // readout TMEM: D_0, D_1 at 0 and NP; scores (64 columns) at RColS; A stages
+  // (stage, block, tile) of 32 columns from RColA
+  static constexpr uint32_t RColS = (2 * NP + 31) / 32 * 32, RColA = RColS + 64;
+  static_assert(RColA + 32 * kRTS * 2 * kRStages <= kRTmemCols, "TMEM budget");
   // readout shared memory
   static constexpr uint32_t RB = NP * kRow;    // NP x 64 snapshot tile
   static constexpr uint32_t RVT = NP * kRow;   // NP x 64-key [V,1]^T block
-  static constexpr uint32_t ROffQ = 0, ROffB = ROffQ + kRTile, ROffK = ROffB + kRBS * kRTS * RB,
+  static constexpr uint32_t ROffQ = 0, ROffB = ROffQ + 2 * kRTile, ROffK = ROffB + kRBS * kRTS * RB,
                             ROffVT = ROffK + kRKB, ROffP = ROffVT + RVT,
                             ROffTiles = ROffP + 2 * kRTile, ROffBar = ROffTiles + kMaxTiles * 8;
   static constexpr uint32_t RSmem = ROffBar + 512 + 1024;  // barriers, TMEM slot, flag
@@ -469,7 +471,7 @@ struct RParams {
   int N, C, nsnap, head0;
   int qk_head0;  // head of group head 0 in the Q / K tensor maps (head0 for the caller's
                  // q, k; 0 for the padded per-group copies)
-  int nblk;      // 128-token blocks per head
+  int npair;     // 256-token pairs of blocks per head
   int cont;      // 1: snapshot slot 0 holds the state before chunk 0
   float *out;    // [BH][N][dV]
   int *err;
@@ -480,6 +482,9 @@ __device__ __forceinline__ float taylor4(float s) {
   return fmaf(fmaf(fmaf(s, 1.0f / 6.0f, 0.5f), s, 1.0f), s, 1.0f);
 }
 
+// One CTA per (head, 256 tokens = two 128-token blocks b of one chunk); the
+// blocks' accumulators D_b[128 x NP] sit side by side in TMEM, so every
+// snapshot tile brought into shared memory feeds the MMAs of both blocks.
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_readout(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -487,6 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                const RParams p) {
   using S = Tc<DK, DV>;
   constexpr int NP = S::NP;
+  constexpr uint32_t ColS = S::RColS, ColA = S::RColA;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   uint8_t *sQ = smem + S::ROffQ, *sB = smem + S::ROffB, *sK = smem + S::ROffK,
@@ -501,16 +507,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert((6 + 2 * kRStages + 2 * kRBS + 2) * 8 <= 512, "barrier region");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // heaviest first: the last 128-token blocks (in the last chunks, with the
+  // heaviest first: the last pairs of blocks (in the last chunks, with the
   // longest in-chunk part) start first, chunk 0 (no inter-chunk part) last
-  const int g_heads = gridDim.x / p.nblk;
-  const int tb = p.nblk - 1 - (int)blockIdx.x / g_heads;
+  const int g_heads = gridDim.x / p.npair;
+  const int tp = p.npair - 1 - (int)blockIdx.x / g_heads;
   const int hrel = (int)blockIdx.x % g_heads;
-  const int t0 = tb * 128;
+  const int t0 = tp * 256;
   const int bh = p.head0 + hrel;
   const int chunk = t0 / p.C;
   const int c0 = chunk * p.C;
-  const int nkb = (t0 - c0) / kKB + 128 / kKB;  // key blocks from the chunk start through t0+127
+  // in-chunk jobs: (block 0, key blocks 0..nkb0-1), then (block 1, 0..nkb1-1)
+  const int nkb0 = (t0 - c0) / kKB + 128 / kKB, nkb1 = nkb0 + 128 / kKB;
+  const int njobs = nkb0 + nkb1;
   const bool inter = chunk > 0 || p.cont != 0;
 
   if (inter)
@@ -538,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tD = tmem, tS = tmem + kRColS;
+  const uint32_t tS = tmem + ColS;
 
   if (warp == 0) {
     // ---------------- TMA producer: snapshot tiles S_(c-1)[NP x 64 rows]
@@ -563,69 +571,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 2) {
-    // ---------------- TMA producer: Q once, then K, [V,1]^T blocks of the chunk
+    // ---------------- TMA producer: Q of both blocks once, then per in-chunk
+    // job the K and [V,1]^T blocks of its 64 keys
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmVT);
       const int qk_head = p.qk_head0 + hrel;
-      mbar_arrive_expect_tx(q_full, kRTile);
+      mbar_arrive_expect_tx(q_full, 2 * kRTile);
       tma_load_3d(sQ, &tmQ, q_full, 0, t0, qk_head);
-      int kb = 0;
-      for (; kb < nkb; ++kb) {
-        if (kb > 0 && !mbar_wait(kv_empty, (kb - 1) & 1, abort_flag, p.err, p.wait_limit)) break;
+      tma_load_3d(sQ + kRTile, &tmQ, q_full, 0, t0 + 128, qk_head);
+      int jb = 0;
+      for (; jb < njobs; ++jb) {
+        const int kb = jb < nkb0 ? jb : jb - nkb0;
+        if (jb > 0 && !mbar_wait(kv_empty, (jb - 1) & 1, abort_flag, p.err, p.wait_limit)) break;
         mbar_arrive_expect_tx(kv_full, kRKB + S::RVT);
         tma_load_3d(sK, &tmK, kv_full, 0, c0 + kKB * kb, qk_head);
         tma_load_3d(sVT, &tmVT, kv_full, c0 + kKB * kb, 0, hrel);
       }
       volatile int never = 0;
       mbar_wait(q_full, 0, &never, p.err);
-      if (kb > 0) mbar_wait(kv_full, (kb - 1) & 1, &never, p.err);
+      if (jb > 0) mbar_wait(kv_full, (jb - 1) & 1, &never, p.err);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_nv = idesc_bf16_f32(128, NP, false, false);  // B: NP rows, K-major
       constexpr uint32_t id_qk = idesc_bf16_f32(128, kKB, false, false);
-      bool d_init = false, ok = true;
-      int kb_qk = 0, kb_pv = 0;
+      bool d_init[2] = {false, false}, ok = true;
+      int jq = 0, jp = 0;  // next job for scores / for P [V, 1]
       const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), vt0 = smem_u32(sVT);
       const uint32_t p0 = smem_u32(sP);
       ok = mbar_wait(q_full, 0, abort_flag, p.err, p.wait_limit);
       // in-chunk part, advanced whenever its inputs are ready
       auto intra = [&](bool block) {
-        while (ok && kb_pv < nkb) {
-          if (kb_qk == kb_pv) {  // next: scores of block kb_qk
+        while (ok && jp < njobs) {
+          if (jq == jp) {  // next: scores of job jq
             if (block) {
-              if (!(ok = mbar_wait(kv_full, kb_qk & 1, abort_flag, p.err, p.wait_limit))) return;
-            } else if (!mbar_test_wait(kv_full, kb_qk & 1)) {
+              if (!(ok = mbar_wait(kv_full, jq & 1, abort_flag, p.err, p.wait_limit))) return;
+            } else if (!mbar_test_wait(kv_full, jq & 1)) {
               return;
             }
             tc_fence_after();
+            const uint32_t qb = q0 + (jq < nkb0 ? 0u : kRTile);
 #pragma unroll
             for (int k = 0; k < DK / 16; ++k)
-              mma_bf16_ss(tS, smem_desc_sw128(q0 + 32 * k, 16, 1024),
+              mma_bf16_ss(tS, smem_desc_sw128(qb + 32 * k, 16, 1024),
                           smem_desc_sw128(k0 + 32 * k, 16, 1024), id_qk, k > 0 ? 1u : 0u);
             mma_commit(s_full);
-            ++kb_qk;
-          } else {  // next: P [V, 1] of block kb_pv
+            ++jq;
+          } else {  // next: P [V, 1] of job jp into its block's accumulator
             if (block) {
-              if (!(ok = mbar_wait(p_full, kb_pv & 1, abort_flag, p.err, p.wait_limit))) return;
-            } else if (!mbar_test_wait(p_full, kb_pv & 1)) {
+              if (!(ok = mbar_wait(p_full, jp & 1, abort_flag, p.err, p.wait_limit))) return;
+            } else if (!mbar_test_wait(p_full, jp & 1)) {
               return;
             }
             tc_fence_after();
+            const int b = jp < nkb0 ? 0 : 1;
 #pragma unroll
             for (int k = 0; k < 2 * (kKB / 16); ++k) {  // hi part, then lo part
               const int kk = k % (kKB / 16);
               const uint64_t ad =
                   smem_desc_sw128(p0 + (k / (kKB / 16)) * kRTile + 32 * kk, 16, 1024);
               const uint64_t bd = smem_desc_sw128(vt0 + 32 * kk, 16, 1024);
-              mma_bf16_ss(tD, ad, bd, id_nv, (d_init || k > 0) ? 1u : 0u);
+              mma_bf16_ss(tmem + b * NP, ad, bd, id_nv, (d_init[b] || k > 0) ? 1u : 0u);
             }
-            d_init = true;
+            d_init[b] = true;
             mma_commit(kv_empty);
-            ++kb_pv;
+            ++jp;
           }
         }
       };
@@ -643,15 +656,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nt = min(kRTS, p.n_tiles - kRTS * i);
           for (int t = 0; t < nt; ++t) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_bf16_ts(tD, tmem + kRColA + (st * kRTS + t) * 32 + 8 * k,
-                          smem_desc_sw128(b0 + (bs * kRTS + t) * S::RB + 32 * k, 16, 1024),
-                          id_nv, (d_init || k > 0) ? 1u : 0u);
-            d_init = true;
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t bd = smem_desc_sw128(b0 + (bs * kRTS + t) * S::RB + 32 * k, 16, 1024);
+              // the two blocks share each B: consecutive MMAs, different D
+#pragma unroll
+              for (int b = 0; b < 2; ++b)
+                mma_bf16_ts(tmem + b * NP, tmem + ColA + ((st * 2 + b) * kRTS + t) * 32 + 8 * k, bd,
+                            id_nv, (d_init[b] || k > 0) ? 1u : 0u);
+            }
+            d_init[0] = d_init[1] = true;
           }
           mma_commit(&a_empty[st]);
           mma_commit(&b_empty[bs]);
-          if (i & 1) intra(false);
+          intra(false);
         }
       }
       if (ok) intra(true);
@@ -666,11 +683,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- epilogue: in-chunk Taylor scores, then normalisation
     const int q4 = warp & 3;
     const int row = 32 * q4 + lane;
-    const int tok = t0 + row;
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
     bool ok = true;
-    for (int kb = 0; ok && kb < nkb; ++kb) {
-      if (!(ok = mbar_wait(s_full, kb & 1, abort_flag, p.err, p.wait_limit))) break;
+    for (int jb = 0; ok && jb < njobs; ++jb) {
+      const int b = jb < nkb0 ? 0 : 1, kb = jb - b * nkb0;
+      const int tok = t0 + 128 * b + row;
+      if (!(ok = mbar_wait(s_full, jb & 1, abort_flag, p.err, p.wait_limit))) break;
       tc_fence_after();
       {
         uint32_t v[kKB];
@@ -702,29 +720,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && (ok = mbar_wait(o_full, 0, abort_flag, p.err, p.wait_limit))) {
       tc_fence_after();
-      uint32_t v[NP];
+      for (int b = 0; b < 2; ++b) {
+        const int tok = t0 + 128 * b + row;
+        uint32_t v[NP];
 #pragma unroll
-      for (int j = 0; j < NP / 16; ++j)
-        tmem_ld16(tD + tl + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
-      tmem_ld_wait();
-      if (tok < p.N) {
-        const float den = __uint_as_float(v[DV]);
-        float4 *dst = reinterpret_cast<float4 *>(p.out + ((size_t)bh * p.N + tok) * DV);
+        for (int j = 0; j < NP / 16; ++j)
+          tmem_ld16(tmem + b * NP + tl + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+        tmem_ld_wait();
+        if (tok < p.N) {
+          const float den = __uint_as_float(v[DV]);
+          float4 *dst = reinterpret_cast<float4 *>(p.out + ((size_t)bh * p.N + tok) * DV);
 #pragma unroll
-        for (int n = 0; n < DV / 4; ++n)
-          dst[n] = make_float4(__uint_as_float(v[4 * n]) / den, __uint_as_float(v[4 * n + 1]) / den,
-                               __uint_as_float(v[4 * n + 2]) / den,
-                               __uint_as_float(v[4 * n + 3]) / den);
+          for (int n = 0; n < DV / 4; ++n)
+            dst[n] = make_float4(__uint_as_float(v[4 * n]) / den, __uint_as_float(v[4 * n + 1]) / den,
+                                 __uint_as_float(v[4 * n + 2]) / den,
+                                 __uint_as_float(v[4 * n + 3]) / den);
+        }
       }
     }
   } else if (warp >= 8 && inter) {
     // ---------------- feature generators: phi(Q) tiles, one thread per token;
-    // the two warps of a TMEM lane quarter split every stage's tiles
+    // warps 8-11 generate block 0, warps 12-15 block 1
     const int gw = warp - 8;
-    const int half = gw >> 2;
+    const int b = gw >> 2;
     const int row = lane + 32 * (gw & 3);
     bool ok = mbar_wait(q_full, 0, abort_flag, p.err, p.wait_limit);
-    const uint8_t *qrow = sQ + row * kRow;
+    const uint8_t *qrow = sQ + b * kRTile + row * kRow;
+    const uint32_t tl = (uint32_t)(32 * (gw & 3)) << 16;
     const int n_stages = (p.n_tiles + kRTS - 1) / kRTS;
     for (int i = 0; ok && i < n_stages; ++i) {
       const int st = i % kRStages;
@@ -732,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             p.err, p.wait_limit)))
         break;
 #pragma unroll 1
-      for (int t = half; t < kRTS; t += 2) {
+      for (int t = 0; t < kRTS; ++t) {
         const int ti = kRTS * i + t;
         uint32_t out[32];
         if (ti < p.n_tiles) {
@@ -742,9 +764,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 0; q < 32; ++q) out[q] = 0u;
         }
-        // this thread's token is TMEM lane `row`; a tile's 64 features are 32
-        // packed columns
-        tmem_st32(tmem + ((uint32_t)(32 * (gw & 3)) << 16) + kRColA + (st * kRTS + t) * 32, out);
+        // this thread's token is TMEM lane `row` of block b; a tile's 64
+        // features are 32 packed columns
+        tmem_st32(tmem + tl + ColA + ((st * 2 + b) * kRTS + t) * 32, out);
       }
       tmem_st_wait();
       if (!(ok = mbar_wait(&b_full[i % kRBS], (i / kRBS) & 1, abort_flag, p.err, p.wait_limit)))
@@ -809,7 +831,7 @@ int launch_tc(const void *q, const void *k, const void *v, float *out, float *st
   // leaves TMEM and costs a snapshot write, while the readout hides the longer
   // in-chunk quadratic part behind its inter-chunk MMAs; 4096 measured fastest
   // of 1024 / 2048 / 4096 at 16384 tokens.
-  const int C = N <= kChunk ? ((N + 127) / 128) * 128 : kChunk;
+  const int C = N <= kChunk ? ((N + 255) / 256) * 256 : kChunk;  // whole readout pairs
   // snapshots: the state before each chunk but the first, plus (continued
   // prefill) the initial state before chunk 0 in slot 0
   const int nsnap = (N + C - 1) / C - 1 + (cont ? 1 : 0);
@@ -851,7 +873,7 @@ int launch_tc(const void *q, const void *k, const void *v, float *out, float *st
   }
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
 
-  const int nblk = (N + 127) / 128;
+  const int npair = (N + 255) / 256;
   GenWeights ones;  // the readout generates unweighted monomials
   ones.w3 = ones.w3h = ones.w3s = ones.w2 = ones.w2h = ones.w1 = 1.f;
   for (int h0 = 0; h0 < BH; h0 += G) {
@@ -901,14 +923,14 @@ int launch_tc(const void *q, const void *k, const void *v, float *out, float *st
     rp.nsnap = nsnap;
     rp.head0 = h0;
     rp.qk_head0 = DK == 64 ? h0 : 0;
-    rp.nblk = nblk;
+    rp.npair = npair;
     rp.cont = cont ? 1 : 0;
     rp.out = out;
     rp.err = err;
     rp.wait_limit = tc_wait_limit();
     if (nsnap == 0) mS = mQ;  // never read: no chunk has a predecessor
     prof_kernel_begin(stream, K_TC_READOUT);
-    tc_readout<DK, DV><<<nblk * g, kThreads, S::RSmem, stream>>>(mQ, mK, mVT, mS, rp);
+    tc_readout<DK, DV><<<npair * g, kThreads, S::RSmem, stream>>>(mQ, mK, mVT, mS, rp);
     prof_kernel_end(stream);
   }
   return cuda_status(cudaGetLastError());
