@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "tokens/sec/GPU (prefill & decode) at d_K=64,P=4; % tensor / HBM roofline"
 PREFILL = dict(B=1, H=8, N=16384, dK=64, dV=64, P=4)
+PREFILL_DK32 = dict(B=4, H=8, N=4096, dK=32, dV=32, P=4)
 DECODE = dict(B=32, H=8, N=8192, dK=64, dV=64, P=4)
 WORKLOAD = ("prefill B=1,H=8,N=16384,dK=dV=64,P=4 bf16 (one sata_prefill per step); "
             "decode B=32,H=8,dK=dV=64,P=4 fp32 state of an N=8192 bf16 prefill "
@@ -56,6 +57,12 @@ def peaks():
 
 def basis_m(dK, P):
     return math.comb(dK + P - 1, P - 1)
+
+
+def alg_one(w, m):
+    """Algorithmic flops of one of the two state contractions for workload w:
+    B*H*N tokens x 2 (dV+1) m."""
+    return w["B"] * w["H"] * w["N"] * 2 * (w["dV"] + 1) * m
 
 
 # --------------------------------------------------------------- clocks sampler
@@ -333,7 +340,10 @@ def run_ours(args, rank, world, local_rank):
         # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
         bound, peak, unit = "alu", 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12, "TFLOP/s"
     achieved = alg / (top_ms / 1e3) / 1e12
+    # both state contractions over the whole step, per GPU
+    step_tflops = 2 * alg_one(w, m) / (total_ms / args.steps / 1e3) / 1e12
     roof = {"bound": bound, "kernel": top, "achieved": achieved, "peak": peak, "unit": unit,
+            "step_tensor_tflops": step_tflops, "step_frac": step_tflops / pk["bf16_tflops"],
             "frac": achieved / peak, "traffic": traffic_record(top),
             "peak_source": pk["source"] if bound == "tensor" else "derived: 148x128x2 flop x sm_max_mhz",
             "kernel_ms": top_ms, "algorithmic_flop_per_launch": alg,
@@ -364,6 +374,56 @@ def run_ours(args, rank, world, local_rank):
            "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (q, k, v)),
            "d2h_bytes_per_step": out.numel() * 4 + state.numel() * 4}
     del qd, kd, vd, out, state, q, k, v, qh, kh, vh, out_h, st_h
+
+    # ---------------- the bf16 dK = dV = 32 prefill workload ([4,8,4096,32])
+    pw3 = PREFILL_DK32
+    m3 = basis_m(pw3["dK"], pw3["P"])
+    q3, k3, v3 = (t.to(dev) for t in make_qkv(pw3["B"], pw3["H"], pw3["N"], pw3["dK"], pw3["dV"],
+                                              seed=20261203 + 1000 * rank, dtype="bf16"))
+    out3 = torch.empty(pw3["B"], pw3["H"], pw3["N"], pw3["dV"], device=dev)
+    st3 = torch.empty(pw3["B"], pw3["H"], m3, pw3["dV"] + 1, device=dev)
+
+    def prefill3():
+        sata.sata_prefill(q3, k3, v3, out3, st3, pw3["B"], pw3["H"], pw3["N"], pw3["dK"],
+                          pw3["dV"], pw3["P"], torch.bfloat16, stream)
+
+    for _ in range(args.warmup):
+        prefill3()
+    torch.cuda.synchronize()
+    sata.sata_profile_enable(True)
+    k3ms, t3 = {}, []
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        prefill3()
+        b.record(stream)
+        for name, ms in sata.sata_profile_read():
+            k3ms.setdefault(name, []).append(ms)
+            launches += 1
+        t3.append(a.elapsed_time(b))
+    torch.cuda.synchronize()
+    barrier()
+    sata.sata_profile_enable(False)
+    tot3 = max_over_ranks(sum(t3))
+    share3 = {n: sum(x) for n, x in k3ms.items()}
+    top3 = max(share3, key=share3.get)
+    top3_ms = statistics.mean(k3ms[top3])
+    alg3 = pw3["B"] * pw3["H"] * pw3["N"] * 2 * (pw3["dV"] + 1) * m3
+    ach3 = alg3 / (top3_ms / 1e3) / 1e12
+    prefill_dk32 = {
+        "workload": "prefill B=4,H=8,N=4096,dK=dV=32,P=4 bf16 (one sata_prefill per step)",
+        "value": weak_scaling_value(world, args.steps, pw3["B"] * pw3["N"], tot3),
+        "unit": "tokens/s", "ms_per_step": tot3 / args.steps,
+        "step_tensor_tflops": 2 * alg3 / (tot3 / args.steps / 1e3) / 1e12,
+        "roofline": {"bound": "tensor", "kernel": top3, "achieved": ach3, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": ach3 / pk["bf16_tflops"],
+                     "peak_source": pk["source"], "kernel_ms": top3_ms,
+                     "algorithmic_flop_per_launch": alg3,
+                     "kernel_share": {n: x / sum(share3.values()) for n, x in share3.items()}},
+    }
+    del q3, k3, v3, out3, st3
 
     # ---------------- decode: fp32 state and mixed-precision state
     dw = DECODE
@@ -476,7 +536,8 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "prefill: 256 MiB L2 flush between timed steps; decode: 3.19 GB fp32 "
                          "(1.66 GB mixed) state > L2",
                    "decode_steps": nsteps},
-        "roofline": roof, "decode": decode, "e2e": e2e, "gpu_launches": launches,
+        "roofline": roof, "decode": decode, "prefill_dk32": prefill_dk32, "e2e": e2e,
+        "gpu_launches": launches,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
