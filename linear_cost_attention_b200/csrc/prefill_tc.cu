@@ -123,13 +123,26 @@ struct UParams {
   const int32_t *grp_row;    // [n_grp][kR][128] lexicographic basis row, -1 padding
   const float *grp_w;        // [n_grp][kR][128] basis weight
   int n_grp;                 // items per head
-  int N, Npad, C, nsnap, m, m_pad, n_items, head0;
+  // Work units: units [0, n_full) are whole items (unit = item index); the
+  // other items are split into two half-items of 2 tiles (unit n_full + 2 h +
+  // x = half x of item n_full + h), so the last round spreads over more CTAs.
+  int n_full, n_units;
+  int N, Npad, C, nsnap, m, m_pad, head0;
   int cont;             // 1: start from the state in `state` (continued prefill)
   __nv_bfloat16 *snap;  // [G][nsnap][dV+1][m_pad]; slot 0 = initial state if cont
   float *state;         // [BH][m][dV+1]
   int *err;
   long long wait_limit;  // cycles before a role's wait gives up (drains: full limit)
 };
+
+struct Unit {
+  int item, f0, nr;  // item, its first tile, tiles in this unit
+};
+__device__ __forceinline__ Unit unit_of(const UParams &p, int u) {
+  if (u < p.n_full) return {u, 0, kR};
+  const int h = u - p.n_full;
+  return {p.n_full + (h >> 1), (h & 1) * (kR / 2), kR / 2};
+}
 
 // One item = (head, kR state tiles of 128 basis rows).  Thread = TMEM lane of
 // all kR tiles: each generator thread owns the kR rows of its lane group
@@ -201,8 +214,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
       prefetch_tensormap(&tmVT);
       uint32_t ik = 0;
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int hb = item / p.n_grp;
+      for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+        const int hb = unit_of(p, u).item / p.n_grp;
         for (int s = 0; s < nK; ++s, ++ik) {
           const int st = ik % kKS;
           if (ik >= kKS && !(ok = mbar_wait(&kv_empty[st], ((ik / kKS) - 1) & 1, abort_flag,
@@ -225,8 +238,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
       uint32_t ia = 0, events = 0, items = 0;
       bool after_event = false;
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items) {
-        if (p.cont) {  // the epilogue has loaded the item's initial state into TMEM
+      for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x, ++items) {
+        const int nr = unit_of(p, u).nr;
+        if (p.cont) {  // the epilogue has loaded the unit's initial state into TMEM
           if (!(ok = mbar_wait(d_ready, items & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
         }
@@ -239,8 +253,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
             break;
           tc_fence_after();
           if (after_event) {
-            // every tile's barrier is waited once per event, in order, so no
-            // barrier can run two phases ahead of its waiter
+            // every tile's barrier is waited once per event, in order (all kR
+            // of them, whatever the unit's width), so no barrier can run two
+            // phases ahead of its waiter
             for (int f = 0; ok && f < kR; ++f)
               ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err, p.wait_limit);
             if (!ok) break;
@@ -254,8 +269,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
             const uint64_t bd = smem_desc_sw128(b0 + 32 * k, 16, 1024);
 #pragma unroll
             for (int f = 0; f < kR; ++f)
-              mma_bf16_ts(tmem + f * NP, tmem + S::UColA + (as * kR + f) * (kAT / 2) + 8 * k, bd,
-                          idesc, (a > 0 || k > 0 || p.cont) ? 1u : 0u);
+              if (f < nr)
+                mma_bf16_ts(tmem + f * NP, tmem + S::UColA + (as * kR + f) * (kAT / 2) + 8 * k,
+                            bd, idesc, (a > 0 || k > 0 || p.cont) ? 1u : 0u);
           }
           after_event = false;
           mma_commit(&a_empty[as]);
@@ -277,14 +293,15 @@ __global__ void __launch_bounds__(kUThreads, 1)
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
     uint32_t events = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int hb = item / p.n_grp, itl = item % p.n_grp;
+    for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+      const Unit un = unit_of(p, u);
+      const int hb = un.item / p.n_grp, itl = un.item % p.n_grp;
       if (p.cont) {
         // continued prefill: S' = S_0 / w into the TMEM tiles (the item's MMAs
         // accumulate onto it), and the snapshot before chunk 0 (slot 0) is
         // w^2 S' = w S_0.  This thread writes the same state rows at the end.
-        for (int f = 0; f < kR; ++f) {
-          const size_t gk = ((size_t)itl * kR + f) * 128 + row;
+        for (int f = 0; f < un.nr; ++f) {
+          const size_t gk = ((size_t)itl * kR + un.f0 + f) * 128 + row;
           const int slot = p.grp_slot[gk], r = p.grp_row[gk];
           const float w = p.grp_w[gk];
           const float *src = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * D1;
@@ -314,7 +331,13 @@ __global__ void __launch_bounds__(kUThreads, 1)
         for (int f = 0; ok && f < kR; ++f) {
           if (!(ok = mbar_wait(&snap_full[f], events & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
-          const size_t gk = ((size_t)itl * kR + f) * 128 + row;
+          if (f >= un.nr) {  // a tile this unit does not use: keep the barriers in step
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&snap_done[f]);
+            continue;
+          }
+          const size_t gk = ((size_t)itl * kR + un.f0 + f) * 128 + row;
           const int slot = p.grp_slot[gk];
           const int r = boundary ? -1 : p.grp_row[gk];
           const float w = p.grp_w[gk];
@@ -356,14 +379,18 @@ __global__ void __launch_bounds__(kUThreads, 1)
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
     uint32_t ia = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int itl = item % p.n_grp;
+    for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+      const Unit un = unit_of(p, u);
+      const int itl = un.item % p.n_grp;
       const uint64_t ix = p.grp_idx[(size_t)itl * 128 + row];
       // byte offset of each factor row inside a K^T box, and its swizzle phase
       const uint32_t rj = (uint32_t)(ix & 0xff), rl = (uint32_t)((ix >> 8) & 0xff);
+      // the unit's tiles f = 0..nr-1 are the item's tiles f0 + f
       uint32_t ri[kR];
 #pragma unroll
-      for (int f = 0; f < kR; ++f) ri[f] = (uint32_t)((ix >> (16 + 8 * f)) & 0xff);
+      for (int f = 0; f < kR; ++f)
+        ri[f] = (uint32_t)((ix >> (16 + 8 * ((un.f0 + f) & (kR - 1)))) & 0xff);
+      const int nr = un.nr;
       for (int a = 0; ok && a < nA; ++a, ++ia) {
         const int as = ia % kAS;
         const uint32_t kv = (ia / 2) % kKS;
@@ -393,6 +420,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
                                      bmul2(xj.w, xl.w));
 #pragma unroll
           for (int f = 0; f < kR; ++f) {
+            if (f >= nr) continue;
             const uint4 xi = lds128(kt + ri[f] * kRow + ((c ^ (ri[f] & 7)) << 4));
             out[f][4 * g8 + 0] = bmul2(xi.x, u.x);
             out[f][4 * g8 + 1] = bmul2(xi.y, u.y);
@@ -402,7 +430,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
         }
 #pragma unroll
         for (int f = 0; f < kR; ++f)
-          tmem_st8(tmem + tl + S::UColA + (as * kR + f) * (kAT / 2) + 8 * hf, out[f]);
+          if (f < nr) tmem_st8(tmem + tl + S::UColA + (as * kR + f) * (kAT / 2) + 8 * hf, out[f]);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -903,7 +931,13 @@ int launch_tc(const void *q, const void *k, const void *v, float *out, float *st
     up.nsnap = nsnap;
     up.m = (int)basis->m;
     up.m_pad = m_pad;
-    up.n_items = g * basis->n_grp;
+    // whole items for full rounds of the grid; the rest as half-items when
+    // they fit in one more round
+    const int n_items = g * basis->n_grp;
+    const int grid = std::min(n_items, nsm);
+    const int rest = n_items % grid;
+    up.n_full = 2 * rest <= grid ? n_items - rest : n_items;
+    up.n_units = up.n_full + 2 * (n_items - up.n_full);
     up.head0 = h0;
     up.cont = cont ? 1 : 0;
     up.snap = snap;
@@ -911,8 +945,7 @@ int launch_tc(const void *q, const void *k, const void *v, float *out, float *st
     up.err = err;
     up.wait_limit = tc_wait_limit();
     prof_kernel_begin(stream, K_TC_CHUNK_STATES);
-    tc_chunk_states<DK, DV><<<std::min(up.n_items, nsm), kUThreads, S::USmem, stream>>>(mKT, mVT,
-                                                                                      up);
+    tc_chunk_states<DK, DV><<<grid, kUThreads, S::USmem, stream>>>(mKT, mVT, up);
     prof_kernel_end(stream);
     RParams rp;
     rp.tiles = reinterpret_cast<const TileDesc *>(basis->tile_desc);
