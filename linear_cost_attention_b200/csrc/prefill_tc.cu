@@ -99,7 +99,7 @@ template <int DK, int DV> struct Tc {
   static constexpr uint32_t UKTh = (KR * kRow + 1023) / 1024 * 1024;
   static constexpr uint32_t UVTh = NP * kRow;
   static constexpr uint32_t UOffKT = 0, UOffVT = kKS * UKTh, UOffBar = UOffVT + kKS * UVTh;
-  static constexpr uint32_t USmem = UOffBar + 256 + 1024;
+  static constexpr uint32_t USmem = UOffBar + 512 + 1024;  // barriers, TMEM slot, flag
   // TMEM: tile f's accumulator at columns f*NP; A stages (kR tiles x 16
   // columns of packed token pairs each) from UColA
   static constexpr uint32_t UColA = (kR * NP + 31) / 32 * 32;
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
            *drain = snap_done + kR, *d_ready = drain + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(d_ready + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(d_ready + 2);
-  static_assert((2 * kKS + 2 * kAS + 2 * kR + 2) * 8 + 8 <= 256, "barrier region");
+  static_assert((2 * kKS + 2 * kAS + 2 * kR + 2) * 8 + 8 <= 512, "barrier region");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
