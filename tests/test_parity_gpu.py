@@ -323,7 +323,7 @@ def test_workload5_decode():
     serr = state_col_error(st_gpu, S_or)
     record("workload 5 (decode B=32,H=8, 1024 steps; heads (3,1),(30,6) every step)",
            out_err=worst, state_err=serr, excluded_rows=0, rows=2 * w.decode_steps,
-           tol=TOL["bf16"], dtype="bfloat16", kernels=["decode_stream", "decode_finalize"])
+           tol=TOL["bf16"], dtype="bfloat16", kernels=launched_kernels())
     assert worst <= TOL["bf16"], worst
     assert serr <= TOL["bf16"]
 
