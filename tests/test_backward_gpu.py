@@ -51,12 +51,14 @@ def test_backward_matches_oracle(B, H, N, dK, dV, P, dt):
     rq, rk, rv = oracle.attention_grad(q, k, v, dout, P)
     tol = TOL[dt]
     errs = {}
+    # a gradient that is exactly zero (P = 1, or a single token whose output
+    # is v_0 whatever q, k are) is compared on the scale of the largest one
+    scale = max(float(np.max(np.abs(r))) for r in (rq, rk, rv))
     for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
         got = got.cpu().double().numpy()
         assert np.isfinite(got).all()
         if np.max(np.abs(ref)) == 0:
-            assert np.all(got == 0), name
-            errs[name] = 0.0
+            errs[name] = float(np.max(np.abs(got))) / scale
             continue
         errs[name] = grad_err(got, ref)
     path = os.environ.get("SATA_PARITY_LOG")
