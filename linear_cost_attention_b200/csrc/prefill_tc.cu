@@ -63,12 +63,12 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 }
 
 // ------------------------------------------------------------ state kernel
-constexpr int kR = kGroupRows;  // 128-row state tiles per item (rows per generator thread)
-constexpr int kAT = 32;         // tokens per A stage (two K-steps of 16)
-constexpr int kAS = 3;          // A stages in TMEM
-constexpr int kKT = 64;         // tokens per K^T / [V,1]^T stage (one TMA box of each)
-constexpr int kKS = 4;          // K^T / [V,1]^T stages in shared memory
-constexpr int kUGenWarps = 8;   // two per TMEM lane quarter, 16 tokens of each A stage each
+constexpr int kT = 2;           // 128-row state tiles per work unit (rows per generator thread)
+constexpr int kAT = 128;        // tokens per A stage (eight K-steps of 16)
+constexpr int kAS = 2;          // A stages in TMEM
+constexpr int kKT = 64;         // tokens per K^T / [V,1]^T box (two boxes per A stage)
+constexpr int kKS = 8;          // K^T / [V,1]^T boxes in shared memory
+constexpr int kUGenWarps = 8;   // two per TMEM lane quarter, one box (64 tokens) each
 constexpr int kUEpiWarp0 = 2, kUGenWarp0 = 6;  // warps 2..5 epilogue, 6.. generators
 constexpr int kUThreads = 32 * (kUGenWarp0 + kUGenWarps);
 constexpr uint32_t kUTmemCols = 512;
@@ -100,10 +100,10 @@ template <int DK, int DV> struct Tc {
   static constexpr uint32_t UVTh = NP * kRow;
   static constexpr uint32_t UOffKT = 0, UOffVT = kKS * UKTh, UOffBar = UOffVT + kKS * UVTh;
   static constexpr uint32_t USmem = UOffBar + 512 + 1024;  // barriers, TMEM slot, flag
-  // TMEM: tile f's accumulator at columns f*NP; A stages (kR tiles x 16
+  // TMEM: tile f's accumulator at columns f*NP; A stages (kT tiles x 64
   // columns of packed token pairs each) from UColA
-  static constexpr uint32_t UColA = (kR * NP + 31) / 32 * 32;
-  static_assert(UColA + kAS * kR * (kAT / 2) <= kUTmemCols, "TMEM budget");
+  static constexpr uint32_t UColA = (kT * NP + 31) / 32 * 32;
+  static_assert(UColA + kAS * kT * (kAT / 2) <= kUTmemCols, "TMEM budget");
   // readout TMEM: D_0, D_1 at 0 and NP; scores (64 columns) at RColS; A stages
   // (stage, block, tile) of 32 columns from RColA
   static constexpr uint32_t RColS = (2 * NP + 31) / 32 * 32, RColA = RColS + 64;
@@ -119,13 +119,14 @@ template <int DK, int DV> struct Tc {
 
 struct UParams {
   const uint64_t *grp_idx;   // [n_grp][128] j | l << 8 | i_f << (16 + 8 f) (dK = the ones row)
-  const int32_t *grp_slot;   // [n_grp][kR][128] tile-order slot (snapshot column), -1 padding
-  const int32_t *grp_row;    // [n_grp][kR][128] lexicographic basis row, -1 padding
-  const float *grp_w;        // [n_grp][kR][128] basis weight
-  int n_grp;                 // items per head
-  // Work units: units [0, n_full) are whole items (unit = item index); the
-  // other items are split into two half-items of 2 tiles (unit n_full + 2 h +
-  // x = half x of item n_full + h), so the last round spreads over more CTAs.
+  const int32_t *grp_slot;   // [n_grp][4][128] tile-order slot (snapshot column), -1 padding
+  const int32_t *grp_row;    // [n_grp][4][128] lexicographic basis row, -1 padding
+  const float *grp_w;        // [n_grp][4][128] basis weight
+  int n_grp;                 // items (lane groups x 4 rows) per head
+  // Work units: a pair unit is two of an item's four 128-row tiles (rows 0-1
+  // or 2-3 of every lane group); units [0, n_full) are pair units (unit u =
+  // pair u), the pairs after them are split into single-tile units so the
+  // last round spreads over more CTAs.
   int n_full, n_units;
   int N, Npad, C, nsnap, m, m_pad, head0;
   int cont;             // 1: start from the state in `state` (continued prefill)
@@ -136,26 +137,27 @@ struct UParams {
 };
 
 struct Unit {
-  int item, f0, nr;  // item, its first tile, tiles in this unit
+  int item, f0, nr;  // item, its first tile (row of the lane groups), tiles in this unit
 };
 __device__ __forceinline__ Unit unit_of(const UParams &p, int u) {
-  if (u < p.n_full) return {u, 0, kR};
-  const int h = u - p.n_full;
-  return {p.n_full + (h >> 1), (h & 1) * (kR / 2), kR / 2};
+  if (u < p.n_full) return {u >> 1, (u & 1) * kT, kT};
+  const int h = u - p.n_full, pair = p.n_full + (h >> 1);
+  return {pair >> 1, (pair & 1) * kT + (h & 1), 1};
 }
 
-// One item = (head, kR state tiles of 128 basis rows).  Thread = TMEM lane of
-// all kR tiles: each generator thread owns the kR rows of its lane group
-// (tile_order.h), which share two factors x_j x_l and differ in the third
-// x_i; per 8 tokens it loads 2 + kR rows of K^T (index dK is a row of ones
-// that is zero past the sequence end) for kR monomials, and stores the
+// One work unit = (head, kT state tiles of 128 basis rows).  Thread = TMEM
+// lane of the unit's tiles: each generator thread owns kT rows of its lane
+// group (tile_order.h), which share two factors x_j x_l and differ in the
+// third x_i; per 8 tokens it loads 2 + kT rows of K^T (index dK is a row of
+// ones that is zero past the sequence end) for kT monomials, and stores the
 // unweighted monomials with tcgen05.st straight into the A operand in TMEM
 // (basis rows x tokens, two tokens per column).  The MMA accumulates
 // S' += m(K)^T [V, 1] with [V, 1]^T as a K-major B operand (rows of V^T plus
-// its ones row; rows dV+1.. are TMA zero fill), the kR tiles' MMAs sharing
-// each B.  The basis weights are applied when S' leaves TMEM: state = w S',
-// snapshot = w^2 S' (the readout then multiplies by the unweighted m(q):
-// sum_a w_a m_a(q) w_a S'_a = phi(q) . S).
+// its ones row; rows dV+1.. are TMA zero fill); each tile's eight MMAs of a
+// stage are issued back to back into its own accumulator (MMAs that switch
+// accumulators run several times slower).  The basis weights are applied
+// when S' leaves TMEM: state = w S', snapshot = w^2 S' (the readout then
+// multiplies by the unweighted m(q): sum_a w_a m_a(q) w_a S'_a = phi(q) . S).
 template <int DK, int DV>
 __global__ void __launch_bounds__(kUThreads, 1)
     tc_chunk_states(const __grid_constant__ CUtensorMap tmKT, const __grid_constant__ CUtensorMap tmVT,
@@ -167,23 +169,23 @@ __global__ void __launch_bounds__(kUThreads, 1)
   uint8_t *sKT = smem + S::UOffKT, *sVT = smem + S::UOffVT;
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S::UOffBar);
   uint64_t *kv_full = bar, *kv_empty = bar + kKS, *a_full = bar + 2 * kKS,
-           *a_empty = a_full + kAS, *snap_full = a_empty + kAS, *snap_done = snap_full + kR,
-           *drain = snap_done + kR, *d_ready = drain + 1;
+           *a_empty = a_full + kAS, *snap_full = a_empty + kAS, *snap_done = snap_full + kT,
+           *drain = snap_done + kT, *d_ready = drain + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(d_ready + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(d_ready + 2);
-  static_assert((2 * kKS + 2 * kAS + 2 * kR + 2) * 8 + 8 <= 512, "barrier region");
+  static_assert((2 * kKS + 2 * kAS + 2 * kT + 2) * 8 + 8 <= 512, "barrier region");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kKS; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], kUGenWarps);
+      mbar_init(&kv_empty[s], kUGenWarps / 2);  // the four warps that read the box
     }
     for (int s = 0; s < kAS; ++s) {
       mbar_init(&a_full[s], kUGenWarps);
       mbar_init(&a_empty[s], 1);
     }
-    for (int f = 0; f < kR; ++f) {
+    for (int f = 0; f < kT; ++f) {
       mbar_init(&snap_full[f], 1);
       mbar_init(&snap_done[f], 4);
     }
@@ -198,9 +200,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // A stage a of an item covers tokens [32 a, 32 a + 32) and reads K/V stage
-  // a / 2; with global counters (ia over all A stages of this CTA) the K/V
-  // stage is ia / 2 because every item has an even number nA of A stages.
+  // A stage a of a unit covers tokens [128 a, 128 a + 128), the K/V boxes
+  // 2 a and 2 a + 1; with global counters (ia over all A stages of this CTA)
+  // the boxes are 2 ia and 2 ia + 1 because every unit has nK = 2 nA boxes.
   const int nA = p.Npad / kAT, nK = p.Npad / kKT;
   const int a_per_chunk = p.C / kAT;
   auto is_event = [&](int a) {
@@ -235,48 +237,56 @@ __global__ void __launch_bounds__(kUThreads, 1)
     // ---------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, NP, false, false);
-      uint32_t ia = 0, events = 0, items = 0;
+      uint32_t ia = 0, events = 0, units = 0;
       bool after_event = false;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x, ++items) {
+      for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x, ++units) {
         const int nr = unit_of(p, u).nr;
         if (p.cont) {  // the epilogue has loaded the unit's initial state into TMEM
-          if (!(ok = mbar_wait(d_ready, items & 1, abort_flag, p.err, p.wait_limit))) break;
+          if (!(ok = mbar_wait(d_ready, units & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
         }
         for (int a = 0; ok && a < nA; ++a, ++ia) {
           const int as = ia % kAS;
-          // a_full also covers kv_full: every generator warp waited on the K/V
-          // stage before arriving.  One barrier wait per A stage: a wait in
-          // this thread stalls until the MMAs already issued have drained.
+          // a_full also covers kv_full: every generator warp waited on its K/V
+          // box before arriving.  One barrier wait per A stage: a wait in this
+          // thread stalls until the MMAs already issued have drained.
           if (!(ok = mbar_wait(&a_full[as], (ia / kAS) & 1, abort_flag, p.err, p.wait_limit)))
             break;
           tc_fence_after();
-          if (after_event) {
-            // every tile's barrier is waited once per event, in order (all kR
-            // of them, whatever the unit's width), so no barrier can run two
-            // phases ahead of its waiter
-            for (int f = 0; ok && f < kR; ++f)
+          const uint32_t vt0 = smem_u32(sVT) + ((2 * ia) % kKS) * S::UVTh;
+          const uint32_t vt1 = smem_u32(sVT) + ((2 * ia + 1) % kKS) * S::UVTh;
+#pragma unroll
+          for (int f = 0; f < kT; ++f) {
+            if (f >= nr) break;
+            if (after_event) {
+              // tile f has been read out at the last event (every tile's
+              // barrier is waited once per event, in order)
+              if (!(ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err,
+                                   p.wait_limit)))
+                break;
+              tc_fence_after();
+            }
+            // the tile's eight MMAs back to back on its own accumulator
+#pragma unroll
+            for (int k = 0; k < kAT / 16; ++k) {
+              const uint64_t bd =
+                  smem_desc_sw128((k < 4 ? vt0 : vt1) + 32 * (k & 3), 16, 1024);
+              mma_bf16_ts(tmem + f * NP, tmem + S::UColA + (as * kT + f) * (kAT / 2) + 8 * k, bd,
+                          idesc, (a > 0 || k > 0 || p.cont) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          if (after_event && nr < kT) {
+            // keep the unused tile's barrier in step
+            for (int f = nr; ok && f < kT; ++f)
               ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err, p.wait_limit);
             if (!ok) break;
-            tc_fence_after();
-          }
-          const uint32_t b0 = smem_u32(sVT + ((ia / 2) % kKS) * S::UVTh) + (ia & 1) * 64;
-          // the kR tiles' MMAs alternate, so consecutive MMAs accumulate into
-          // different TMEM columns and share their B operand
-#pragma unroll
-          for (int k = 0; k < kAT / 16; ++k) {
-            const uint64_t bd = smem_desc_sw128(b0 + 32 * k, 16, 1024);
-#pragma unroll
-            for (int f = 0; f < kR; ++f)
-              if (f < nr)
-                mma_bf16_ts(tmem + f * NP, tmem + S::UColA + (as * kR + f) * (kAT / 2) + 8 * k,
-                            bd, idesc, (a > 0 || k > 0 || p.cont) ? 1u : 0u);
           }
           after_event = false;
           mma_commit(&a_empty[as]);
           if (is_event(a)) {
-            for (int f = 0; f < kR; ++f) mma_commit(&snap_full[f]);
+            for (int f = 0; f < kT; ++f) mma_commit(&snap_full[f]);
             ++events;
             after_event = true;
           }
@@ -297,11 +307,11 @@ __global__ void __launch_bounds__(kUThreads, 1)
       const Unit un = unit_of(p, u);
       const int hb = un.item / p.n_grp, itl = un.item % p.n_grp;
       if (p.cont) {
-        // continued prefill: S' = S_0 / w into the TMEM tiles (the item's MMAs
+        // continued prefill: S' = S_0 / w into the TMEM tiles (the unit's MMAs
         // accumulate onto it), and the snapshot before chunk 0 (slot 0) is
         // w^2 S' = w S_0.  This thread writes the same state rows at the end.
         for (int f = 0; f < un.nr; ++f) {
-          const size_t gk = ((size_t)itl * kR + un.f0 + f) * 128 + row;
+          const size_t gk = ((size_t)itl * kGroupRows + un.f0 + f) * 128 + row;
           const int slot = p.grp_slot[gk], r = p.grp_row[gk];
           const float w = p.grp_w[gk];
           const float *src = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * D1;
@@ -328,7 +338,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
         if (!is_event(a)) continue;
         const bool boundary = a != nA - 1;
         const int c = boundary ? (a + 1) / a_per_chunk - 1 + p.cont : 0;
-        for (int f = 0; ok && f < kR; ++f) {
+        for (int f = 0; ok && f < kT; ++f) {
           if (!(ok = mbar_wait(&snap_full[f], events & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
           if (f >= un.nr) {  // a tile this unit does not use: keep the barriers in step
@@ -337,43 +347,42 @@ __global__ void __launch_bounds__(kUThreads, 1)
             if (lane == 0) mbar_arrive(&snap_done[f]);
             continue;
           }
-          const size_t gk = ((size_t)itl * kR + un.f0 + f) * 128 + row;
+          const size_t gk = ((size_t)itl * kGroupRows + un.f0 + f) * 128 + row;
           const int slot = p.grp_slot[gk];
           const int r = boundary ? -1 : p.grp_row[gk];
           const float w = p.grp_w[gk];
           const float scale = boundary ? w * w : w;
-          __nv_bfloat16 *sdst = p.snap + ((size_t)(hb * p.nsnap + c) * D1) * p.m_pad + slot;
-          float *tdst = p.state + ((size_t)(p.head0 + hb) * p.m + (r < 0 ? 0 : r)) * D1;
-          // 16 columns at a time: read, then store; the tile is released once
-          // every column has been read
+          // read the whole tile, release it to the MMAs, then store
+          uint32_t v[NP];
 #pragma unroll
-          for (int j = 0; j < NP / 16; ++j) {
-            uint32_t v[16];
-            tmem_ld16(tmem + tl + f * NP + 16 * j, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int n = 16 * j + e;
-              if (n >= D1) continue;
-              const float x = scale * __uint_as_float(v[e]);
-              if (boundary) {
-                if (slot >= 0) sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(x);
-              } else if (r >= 0) {
-                tdst[n] = x;
-              }
-            }
-          }
+          for (int j = 0; j < NP / 16; ++j)
+            tmem_ld16(tmem + tl + f * NP + 16 * j, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * j]));
+          tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&snap_done[f]);
+          if (boundary) {
+            if (slot >= 0) {
+              __nv_bfloat16 *sdst = p.snap + ((size_t)(hb * p.nsnap + c) * D1) * p.m_pad + slot;
+#pragma unroll
+              for (int n = 0; n < D1; ++n)
+                sdst[(size_t)n * p.m_pad] = __float2bfloat16_rn(scale * __uint_as_float(v[n]));
+            }
+          } else if (r >= 0) {
+            float *tdst = p.state + ((size_t)(p.head0 + hb) * p.m + r) * D1;
+#pragma unroll
+            for (int n = 0; n < D1; ++n) tdst[n] = scale * __uint_as_float(v[n]);
+          }
         }
         ++events;
       }
     }
   } else {
-    // ---------------- generators: one TMEM lane (lane group of kR rows) per thread
+    // ---------------- generators: one TMEM lane (kT rows of a lane group) per
+    // thread; warps 6-9 make tokens [0, 64) of every A stage, warps 10-13
+    // tokens [64, 128), each from its own K^T box
     const int gw = warp - kUGenWarp0;
-    const int hf = gw >> 2;             // tokens [16 hf, 16 hf + 16) of every A stage
+    const int hf = gw >> 2;
     const int q4 = warp & 3;            // TMEM lane quarter
     const int row = 32 * q4 + lane;     // TMEM lane
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
@@ -383,54 +392,49 @@ __global__ void __launch_bounds__(kUThreads, 1)
       const Unit un = unit_of(p, u);
       const int itl = un.item % p.n_grp;
       const uint64_t ix = p.grp_idx[(size_t)itl * 128 + row];
-      // byte offset of each factor row inside a K^T box, and its swizzle phase
       const uint32_t rj = (uint32_t)(ix & 0xff), rl = (uint32_t)((ix >> 8) & 0xff);
-      // the unit's tiles f = 0..nr-1 are the item's tiles f0 + f
-      uint32_t ri[kR];
+      // the unit's tiles f = 0..nr-1 are rows f0 + f of the lane group
+      uint32_t ri[kT];
 #pragma unroll
-      for (int f = 0; f < kR; ++f)
-        ri[f] = (uint32_t)((ix >> (16 + 8 * ((un.f0 + f) & (kR - 1)))) & 0xff);
+      for (int f = 0; f < kT; ++f)
+        ri[f] = (uint32_t)((ix >> (16 + 8 * ((un.f0 + f) & (kGroupRows - 1)))) & 0xff);
       const int nr = un.nr;
       for (int a = 0; ok && a < nA; ++a, ++ia) {
         const int as = ia % kAS;
-        const uint32_t kv = (ia / 2) % kKS;
-        if ((ia & 1) == 0 &&
-            !(ok = mbar_wait(&kv_full[kv], ((ia / 2) / kKS) & 1, abort_flag, p.err, p.wait_limit)))
+        const uint32_t box = 2 * ia + hf;   // this warp's K/V box (global counter)
+        const uint32_t kv = box % kKS;
+        if (!(ok = mbar_wait(&kv_full[kv], (box / kKS) & 1, abort_flag, p.err, p.wait_limit)))
           break;
         if (ia >= kAS) {
           if (!(ok = mbar_wait(&a_empty[as], ((ia / kAS) - 1) & 1, abort_flag, p.err,
                                p.wait_limit)))
             break;
-          // the MMAs of A stage ia - kAS are complete; when that was the second
-          // A stage of its K/V stage, this warp releases the K/V stage
-          const uint32_t done = ia - kAS;
-          if (done & 1) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&kv_empty[(done / 2) % kKS]);
-          }
+          // the MMAs of A stage ia - kAS are complete: its box of this half
+          // can be reloaded
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&kv_empty[(2 * (ia - kAS) + hf) % kKS]);
         }
         const uint32_t kt = smem_u32(sKT) + kv * S::UKTh;
-        uint32_t out[kR][8];
+        uint32_t out[kT][32];
 #pragma unroll
-        for (int g8 = 0; g8 < 2; ++g8) {  // 8 tokens per 16-byte chunk of a K^T row
-          const uint32_t c = (ia & 1) * 4 + hf * 2 + g8;
-          const uint4 xj = lds128(kt + rj * kRow + ((c ^ (rj & 7)) << 4));
-          const uint4 xl = lds128(kt + rl * kRow + ((c ^ (rl & 7)) << 4));
-          const uint4 u = make_uint4(bmul2(xj.x, xl.x), bmul2(xj.y, xl.y), bmul2(xj.z, xl.z),
-                                     bmul2(xj.w, xl.w));
+        for (int c = 0; c < 8; ++c) {  // 8 tokens per 16-byte chunk of a K^T row
+          const uint4 xj = lds128(kt + rj * kRow + (((uint32_t)c ^ (rj & 7)) << 4));
+          const uint4 xl = lds128(kt + rl * kRow + (((uint32_t)c ^ (rl & 7)) << 4));
+          const uint4 pr = make_uint4(bmul2(xj.x, xl.x), bmul2(xj.y, xl.y), bmul2(xj.z, xl.z),
+                                      bmul2(xj.w, xl.w));
 #pragma unroll
-          for (int f = 0; f < kR; ++f) {
+          for (int f = 0; f < kT; ++f) {
             if (f >= nr) continue;
-            const uint4 xi = lds128(kt + ri[f] * kRow + ((c ^ (ri[f] & 7)) << 4));
-            out[f][4 * g8 + 0] = bmul2(xi.x, u.x);
-            out[f][4 * g8 + 1] = bmul2(xi.y, u.y);
-            out[f][4 * g8 + 2] = bmul2(xi.z, u.z);
-            out[f][4 * g8 + 3] = bmul2(xi.w, u.w);
+            const uint4 xi = lds128(kt + ri[f] * kRow + (((uint32_t)c ^ (ri[f] & 7)) << 4));
+            out[f][4 * c + 0] = bmul2(xi.x, pr.x);
+            out[f][4 * c + 1] = bmul2(xi.y, pr.y);
+            out[f][4 * c + 2] = bmul2(xi.z, pr.z);
+            out[f][4 * c + 3] = bmul2(xi.w, pr.w);
           }
         }
 #pragma unroll
-        for (int f = 0; f < kR; ++f)
-          if (f < nr) tmem_st8(tmem + tl + S::UColA + (as * kR + f) * (kAT / 2) + 8 * hf, out[f]);
+        for (int f = 0; f < kT; ++f)
+          if (f < nr) tmem_st32(tmem + tl + S::UColA + (as * kT + f) * (kAT / 2) + 32 * hf, out[f]);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -682,18 +686,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           tc_fence_after();
           const int nt = min(kRTS, p.n_tiles - kRTS * i);
-          for (int t = 0; t < nt; ++t) {
+          // each block's MMAs back to back on its own accumulator (MMAs that
+          // switch accumulators run several times slower); both read the
+          // stage's snapshot tiles
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t bd = smem_desc_sw128(b0 + (bs * kRTS + t) * S::RB + 32 * k, 16, 1024);
-              // the two blocks share each B: consecutive MMAs, different D
+          for (int b = 0; b < 2; ++b) {
+            for (int t = 0; t < nt; ++t) {
 #pragma unroll
-              for (int b = 0; b < 2; ++b)
-                mma_bf16_ts(tmem + b * NP, tmem + ColA + ((st * 2 + b) * kRTS + t) * 32 + 8 * k, bd,
-                            id_nv, (d_init[b] || k > 0) ? 1u : 0u);
+              for (int k = 0; k < 4; ++k)
+                mma_bf16_ts(tmem + b * NP, tmem + ColA + ((st * 2 + b) * kRTS + t) * 32 + 8 * k,
+                            smem_desc_sw128(b0 + (bs * kRTS + t) * S::RB + 32 * k, 16, 1024),
+                            id_nv, (d_init[b] || t > 0 || k > 0) ? 1u : 0u);
             }
-            d_init[0] = d_init[1] = true;
           }
+          d_init[0] = d_init[1] = true;
           mma_commit(&a_empty[st]);
           mma_commit(&b_empty[bs]);
           intra(false);
@@ -931,13 +937,13 @@ int launch_tc(const void *q, const void *k, const void *v, float *out, float *st
     up.nsnap = nsnap;
     up.m = (int)basis->m;
     up.m_pad = m_pad;
-    // whole items for full rounds of the grid; the rest as half-items when
+    // pair units for full rounds of the grid; the rest as single tiles when
     // they fit in one more round
-    const int n_items = g * basis->n_grp;
-    const int grid = std::min(n_items, nsm);
-    const int rest = n_items % grid;
-    up.n_full = 2 * rest <= grid ? n_items - rest : n_items;
-    up.n_units = up.n_full + 2 * (n_items - up.n_full);
+    const int n_pairs = 2 * g * basis->n_grp;
+    const int grid = std::min(n_pairs, nsm);
+    const int rest = n_pairs % grid;
+    up.n_full = 2 * rest <= grid ? n_pairs - rest : n_pairs;
+    up.n_units = up.n_full + 2 * (n_pairs - up.n_full);
     up.head0 = h0;
     up.cont = cont ? 1 : 0;
     up.snap = snap;
