@@ -595,6 +595,14 @@ def profile_case(case: str):
         for t in range(5):
             qt, kt, vt = (x[:, :, t].contiguous().cuda() for x in (q, k, v))
             sata.decode_step(qt, kt, vt, state, P)
+    elif case == "decode_mixed":
+        B, H, N, d, P = 8, 8, 256, 64, 4          # mixed state 415 MB (> L2)
+        q, k, v = make_qkv(B, H, N, d, d, seed=3, dtype="bf16")
+        _, state = sata.prefill(q.cuda(), k.cuda(), v.cuda(), P)
+        lo, hi = sata.split_state(state, P)
+        for t in range(5):
+            qt, kt, vt = (x[:, :, t].contiguous().cuda() for x in (q, k, v))
+            sata.decode_step_mixed(qt, kt, vt, lo, hi, P)
     elif case == "prefill":
         B, H, N, d, P = 1, 2, 8192, 64, 4         # one chunk-boundary snapshot per head
         q, k, v = make_qkv(B, H, N, d, d, seed=4, dtype="bf16")
@@ -623,7 +631,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--ref-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["decode", "prefill", "prefill_full"], default=None,
+    ap.add_argument("--profile-case", choices=["decode", "decode_mixed", "prefill", "prefill_full"],
+                    default=None,
                     help="run a small case of one kernel for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:
