@@ -10,15 +10,15 @@
 //     operand of the state MMAs and of the in-chunk P [V, 1] MMAs.  For
 //     dK = 32 it also writes Q and K padded to 64 columns with zeros, so that
 //     every tile keeps the 128-byte-swizzled layout of 64-element rows.
-//   tc_chunk_states  persistent CTAs (448 threads) over items = (head, four
-//     128-row state tiles); the tiles S'[128 x NP] (dV+1 columns padded to
-//     the MMA's N = NP, a multiple of 16) stay in TMEM for the whole sequence.
-//     Warp 0 brings 64-token K^T and [V,1]^T boxes by TMA; warps 6-13 (one
-//     TMEM lane = one lane group of four basis rows sharing two factors per
-//     thread, tile_order.h) multiply K^T rows for every token and store the
-//     unweighted monomials into a TMEM A stage of 32 tokens; warp 1 (one
-//     thread) issues 8 MMAs M = 128, N = NP, K = 16 per stage (A from TMEM, B
-//     from shared memory), the four tiles alternating on each B.  At each
+//   tc_chunk_states  persistent CTAs (480 threads) over work units = (head,
+//     two 128-row state tiles); the tiles S'[128 x NP] (dV+1 columns padded
+//     to the MMA's N = NP, a multiple of 16) stay in TMEM for the whole
+//     sequence.  Warp 0 brings 64-token K^T and [V,1]^T boxes by TMA; warps
+//     6-13 (one TMEM lane = one lane group of basis rows sharing two factors,
+//     tile_order.h) multiply K^T rows for every token and store the
+//     unweighted monomials into TMEM A stages of 128 tokens; warps 1 and 14
+//     (one thread each, one per tile) issue the tile's 8 MMAs M = 128,
+//     N = NP, K = 16 per stage (A from TMEM, B from shared memory).  At each
 //     chunk boundary warps 2-5 copy w^2 S' into a bf16 snapshot (the state
 //     before the next chunk, "恒定计算成本的工程实现": the fixed-size state);
 //     after the last token they write w S' as the fp32 state in lexicographic
@@ -36,7 +36,7 @@
 //     P_lo [V, 1] into D; out = D[:, :dV] / D[:, dV].  Warp 2 brings Q and the
 //     chunk's K, [V, 1]^T blocks by TMA.
 //
-// The MMA-issuing thread waits on one barrier per stage: a wait there stalls
+// An MMA-issuing thread waits on one barrier per stage: a wait there stalls
 // the tensor pipe, whose queue holds only a couple of MMAs.  Every mbarrier
 // wait is bounded (tc_common.cuh); on a timeout the kernel records an error,
 // drains what it issued and frees its TMEM before returning.
@@ -69,8 +69,9 @@ constexpr int kAS = 2;          // A stages in TMEM
 constexpr int kKT = 64;         // tokens per K^T / [V,1]^T box (two boxes per A stage)
 constexpr int kKS = 8;          // K^T / [V,1]^T boxes in shared memory
 constexpr int kUGenWarps = 8;   // two per TMEM lane quarter, one box (64 tokens) each
-constexpr int kUEpiWarp0 = 2, kUGenWarp0 = 6;  // warps 2..5 epilogue, 6.. generators
-constexpr int kUThreads = 32 * (kUGenWarp0 + kUGenWarps);
+constexpr int kUEpiWarp0 = 2, kUGenWarp0 = 6;  // warps 2..5 epilogue, 6..13 generators
+constexpr int kUMmaWarp1 = kUGenWarp0 + kUGenWarps;  // second MMA issuer (the first is warp 1)
+constexpr int kUThreads = 32 * (kUMmaWarp1 + 1);
 constexpr uint32_t kUTmemCols = 512;
 constexpr int kMaxDevices = 64;  // per-device launch attributes
 constexpr int kChunk = 4096;     // tokens per chunk (a multiple of the 128-token padding)
@@ -170,10 +171,11 @@ __global__ void __launch_bounds__(kUThreads, 1)
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S::UOffBar);
   uint64_t *kv_full = bar, *kv_empty = bar + kKS, *a_full = bar + 2 * kKS,
            *a_empty = a_full + kAS, *snap_full = a_empty + kAS, *snap_done = snap_full + kT,
-           *drain = snap_done + kT, *d_ready = drain + 1;
+           *drain = snap_done + kT, *d_ready = drain + kT;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(d_ready + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(d_ready + 2);
-  static_assert((2 * kKS + 2 * kAS + 2 * kT + 2) * 8 + 8 <= 512, "barrier region");
+  static_assert((2 * kKS + 2 * kAS + 3 * kT + 1) * 8 + 8 <= 512, "barrier region");
+  static_assert(kT == 2, "one MMA-issuing warp per state tile");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -183,13 +185,13 @@ __global__ void __launch_bounds__(kUThreads, 1)
     }
     for (int s = 0; s < kAS; ++s) {
       mbar_init(&a_full[s], kUGenWarps);
-      mbar_init(&a_empty[s], 1);
+      mbar_init(&a_empty[s], kT);  // one commit per MMA issuer
     }
     for (int f = 0; f < kT; ++f) {
       mbar_init(&snap_full[f], 1);
       mbar_init(&snap_done[f], 4);
+      mbar_init(&drain[f], 1);
     }
-    mbar_init(drain, 1);
     mbar_init(d_ready, 4);
     *abort_flag = 0;
     fence_barrier_init();
@@ -233,15 +235,19 @@ __global__ void __launch_bounds__(kUThreads, 1)
         mbar_wait(&kv_full[j % kKS], (j / kKS) & 1, &never, p.err);
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer
+  } else if (warp == 1 || warp == kUMmaWarp1) {
+    // ---------------- MMA issuers: warp 1 issues tile 0's MMAs, the last warp
+    // tile 1's (one thread issues an MMA only every ~60 cycles once the
+    // descriptors change from MMA to MMA, an M = 128, N = 80 MMA takes 40)
     if (lane == 0) {
+      const int f = warp == 1 ? 0 : 1;
       constexpr uint32_t idesc = idesc_bf16_f32(128, NP, false, false);
+      const uint32_t d_tile = tmem + f * NP;
       uint32_t ia = 0, events = 0, units = 0;
       bool after_event = false;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x, ++units) {
-        const int nr = unit_of(p, u).nr;
+        const bool active = f < unit_of(p, u).nr;  // a single-tile unit leaves tile 1 idle
         if (p.cont) {  // the epilogue has loaded the unit's initial state into TMEM
           if (!(ok = mbar_wait(d_ready, units & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
@@ -249,52 +255,42 @@ __global__ void __launch_bounds__(kUThreads, 1)
         for (int a = 0; ok && a < nA; ++a, ++ia) {
           const int as = ia % kAS;
           // a_full also covers kv_full: every generator warp waited on its K/V
-          // box before arriving.  One barrier wait per A stage: a wait in this
-          // thread stalls until the MMAs already issued have drained.
+          // box before arriving
           if (!(ok = mbar_wait(&a_full[as], (ia / kAS) & 1, abort_flag, p.err, p.wait_limit)))
             break;
+          if (after_event) {
+            // the tile has been read out at the last event (waited even when
+            // idle, to keep the barrier in step)
+            if (!(ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err,
+                                 p.wait_limit)))
+              break;
+            after_event = false;
+          }
           tc_fence_after();
-          const uint32_t vt0 = smem_u32(sVT) + ((2 * ia) % kKS) * S::UVTh;
-          const uint32_t vt1 = smem_u32(sVT) + ((2 * ia + 1) % kKS) * S::UVTh;
-#pragma unroll
-          for (int f = 0; f < kT; ++f) {
-            if (f >= nr) break;
-            if (after_event) {
-              // tile f has been read out at the last event (every tile's
-              // barrier is waited once per event, in order)
-              if (!(ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err,
-                                   p.wait_limit)))
-                break;
-              tc_fence_after();
-            }
-            // the tile's eight MMAs back to back on its own accumulator
+          if (active) {
+            const uint32_t vt0 = smem_u32(sVT) + ((2 * ia) % kKS) * S::UVTh;
+            const uint32_t vt1 = smem_u32(sVT) + ((2 * ia + 1) % kKS) * S::UVTh;
+            const uint32_t a_tile = tmem + S::UColA + (as * kT + f) * (kAT / 2);
+            const uint32_t acc0 = (a > 0 || p.cont) ? 1u : 0u;
+            // the tile's eight MMAs back to back on its accumulator
 #pragma unroll
             for (int k = 0; k < kAT / 16; ++k) {
               const uint64_t bd =
                   smem_desc_sw128((k < 4 ? vt0 : vt1) + 32 * (k & 3), 16, 1024);
-              mma_bf16_ts(tmem + f * NP, tmem + S::UColA + (as * kT + f) * (kAT / 2) + 8 * k, bd,
-                          idesc, (a > 0 || k > 0 || p.cont) ? 1u : 0u);
+              mma_bf16_ts(d_tile, a_tile + 8 * k, bd, idesc, k > 0 ? 1u : acc0);
             }
           }
-          if (!ok) break;
-          if (after_event && nr < kT) {
-            // keep the unused tile's barrier in step
-            for (int f = nr; ok && f < kT; ++f)
-              ok = mbar_wait(&snap_done[f], (events - 1) & 1, abort_flag, p.err, p.wait_limit);
-            if (!ok) break;
-          }
-          after_event = false;
           mma_commit(&a_empty[as]);
           if (is_event(a)) {
-            for (int f = 0; f < kT; ++f) mma_commit(&snap_full[f]);
+            mma_commit(&snap_full[f]);
             ++events;
             after_event = true;
           }
         }
       }
-      mma_commit(drain);
+      mma_commit(&drain[f]);
       volatile int never = 0;
-      mbar_wait(drain, 0, &never, p.err);
+      mbar_wait(&drain[f], 0, &never, p.err);
     }
   } else if (warp >= kUEpiWarp0 && warp < kUGenWarp0) {
     // ---------------- epilogue: S' -> snapshot (w^2 S') or state (w S')
