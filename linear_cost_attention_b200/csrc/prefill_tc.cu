@@ -268,17 +268,19 @@ __global__ void __launch_bounds__(kUThreads, 1)
           }
           tc_fence_after();
           if (active) {
-            const uint32_t vt0 = smem_u32(sVT) + ((2 * ia) % kKS) * S::UVTh;
-            const uint32_t vt1 = smem_u32(sVT) + ((2 * ia + 1) % kKS) * S::UVTh;
+            // B descriptors of the stage's two boxes; a K-step of 16 tokens
+            // advances the start address by 32 bytes (2 in the >> 4 field)
+            const uint64_t bd0 =
+                smem_desc_sw128(smem_u32(sVT) + ((2 * ia) % kKS) * S::UVTh, 16, 1024);
+            const uint64_t bd1 =
+                smem_desc_sw128(smem_u32(sVT) + ((2 * ia + 1) % kKS) * S::UVTh, 16, 1024);
             const uint32_t a_tile = tmem + S::UColA + (as * kT + f) * (kAT / 2);
             const uint32_t acc0 = (a > 0 || p.cont) ? 1u : 0u;
             // the tile's eight MMAs back to back on its accumulator
 #pragma unroll
-            for (int k = 0; k < kAT / 16; ++k) {
-              const uint64_t bd =
-                  smem_desc_sw128((k < 4 ? vt0 : vt1) + 32 * (k & 3), 16, 1024);
-              mma_bf16_ts(d_tile, a_tile + 8 * k, bd, idesc, k > 0 ? 1u : acc0);
-            }
+            for (int k = 0; k < kAT / 16; ++k)
+              mma_bf16_ts(d_tile, a_tile + 8 * k, (k < 4 ? bd0 : bd1) + 2 * (k & 3), idesc,
+                          k > 0 ? 1u : acc0);
           }
           mma_commit(&a_empty[as]);
           if (is_event(a)) {
@@ -388,12 +390,16 @@ __global__ void __launch_bounds__(kUThreads, 1)
       const Unit un = unit_of(p, u);
       const int itl = un.item % p.n_grp;
       const uint64_t ix = p.grp_idx[(size_t)itl * 128 + row];
-      const uint32_t rj = (uint32_t)(ix & 0xff), rl = (uint32_t)((ix >> 8) & 0xff);
+      // byte offsets of the factor rows in a K^T box with the row's 128-byte
+      // swizzle of chunk 0 folded in: chunk c of row r sits at
+      // box + (r * 128 + (r % 8) * 16) ^ (c * 16) (boxes are 1024-byte aligned)
+      auto row_off = [](uint32_t r) { return r * kRow + ((r & 7) << 4); };
+      const uint32_t oj = row_off((uint32_t)(ix & 0xff)), ol = row_off((uint32_t)((ix >> 8) & 0xff));
       // the unit's tiles f = 0..nr-1 are rows f0 + f of the lane group
-      uint32_t ri[kT];
+      uint32_t oi[kT];
 #pragma unroll
       for (int f = 0; f < kT; ++f)
-        ri[f] = (uint32_t)((ix >> (16 + 8 * ((un.f0 + f) & (kGroupRows - 1)))) & 0xff);
+        oi[f] = row_off((uint32_t)((ix >> (16 + 8 * ((un.f0 + f) & (kGroupRows - 1)))) & 0xff));
       const int nr = un.nr;
       for (int a = 0; ok && a < nA; ++a, ++ia) {
         const int as = ia % kAS;
@@ -411,26 +417,54 @@ __global__ void __launch_bounds__(kUThreads, 1)
           if (lane == 0) mbar_arrive(&kv_empty[(2 * (ia - kAS) + hf) % kKS]);
         }
         const uint32_t kt = smem_u32(sKT) + kv * S::UKTh;
+        const uint32_t aj = kt + oj, al = kt + ol;
+        uint32_t ai[kT];
+#pragma unroll
+        for (int f = 0; f < kT; ++f) ai[f] = kt + oi[f];
+        const uint32_t tcol = tmem + tl + S::UColA + as * kT * (kAT / 2) + 32 * hf;
+        // 8 tokens per 16-byte chunk of a K^T row; the loads of chunk c + 1
+        // are issued before the products of chunk c, and each half of the 64
+        // tokens goes to TMEM as soon as it is complete
+        uint4 xj = lds128(aj), xl = lds128(al), xi[kT];
+#pragma unroll
+        for (int f = 0; f < kT; ++f)
+          if (f < nr) xi[f] = lds128(ai[f]);
         uint32_t out[kT][32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {  // 8 tokens per 16-byte chunk of a K^T row
-          const uint4 xj = lds128(kt + rj * kRow + (((uint32_t)c ^ (rj & 7)) << 4));
-          const uint4 xl = lds128(kt + rl * kRow + (((uint32_t)c ^ (rl & 7)) << 4));
+        for (int c = 0; c < 8; ++c) {
+          uint4 nj, nl, ni[kT];
+          if (c < 7) {
+            const uint32_t sw = (uint32_t)(c + 1) << 4;
+            nj = lds128(aj ^ sw);
+            nl = lds128(al ^ sw);
+#pragma unroll
+            for (int f = 0; f < kT; ++f)
+              if (f < nr) ni[f] = lds128(ai[f] ^ sw);
+          }
           const uint4 pr = make_uint4(bmul2(xj.x, xl.x), bmul2(xj.y, xl.y), bmul2(xj.z, xl.z),
                                       bmul2(xj.w, xl.w));
 #pragma unroll
           for (int f = 0; f < kT; ++f) {
             if (f >= nr) continue;
-            const uint4 xi = lds128(kt + ri[f] * kRow + (((uint32_t)c ^ (ri[f] & 7)) << 4));
-            out[f][4 * c + 0] = bmul2(xi.x, pr.x);
-            out[f][4 * c + 1] = bmul2(xi.y, pr.y);
-            out[f][4 * c + 2] = bmul2(xi.z, pr.z);
-            out[f][4 * c + 3] = bmul2(xi.w, pr.w);
+            out[f][4 * c + 0] = bmul2(xi[f].x, pr.x);
+            out[f][4 * c + 1] = bmul2(xi[f].y, pr.y);
+            out[f][4 * c + 2] = bmul2(xi[f].z, pr.z);
+            out[f][4 * c + 3] = bmul2(xi[f].w, pr.w);
+          }
+          if (c == 3 || c == 7) {
+#pragma unroll
+            for (int f = 0; f < kT; ++f)
+              if (f < nr)
+                tmem_st16(tcol + f * (kAT / 2) + (c == 3 ? 0 : 16),
+                          *reinterpret_cast<const uint32_t(*)[16]>(&out[f][c == 3 ? 0 : 16]));
+          }
+          if (c < 7) {
+            xj = nj;
+            xl = nl;
+#pragma unroll
+            for (int f = 0; f < kT; ++f) xi[f] = ni[f];
           }
         }
-#pragma unroll
-        for (int f = 0; f < kT; ++f)
-          if (f < nr) tmem_st32(tmem + tl + S::UColA + (as * kT + f) * (kAT / 2) + 32 * hf, out[f]);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
