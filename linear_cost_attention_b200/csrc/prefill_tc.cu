@@ -24,17 +24,19 @@
 //     after the last token they write w S' as the fp32 state in lexicographic
 //     row order.  A continued prefill first loads S_0 / w into the tiles and
 //     S_0 w as snapshot 0.
-//   tc_readout       one CTA (512 threads) per (head, 128 tokens), launched
-//     heaviest first (later chunks first, chunk 0 last):
-//     D[128 x NP] in TMEM accumulates phi(Q) S_(c-1) over the tiles of 64
-//     basis rows (warps 8-15, one thread per token = TMEM lane, generate the
-//     tiles' monomials into TMEM A stages; warp 0 streams the snapshot tiles by
-//     TMA) plus the in-chunk part sum_{c0 <= j <= i} T_4(s_ij) [v_j, 1] per
-//     64-key block: scores Q K^T into TMEM, T_4 and the causal mask by the
-//     epilogue warps 4-7, P split into bf16 hi + lo parts (T_4 rounded to bf16
-//     loses too much on rows whose denominator cancels), P_hi [V, 1] +
-//     P_lo [V, 1] into D; out = D[:, :dV] / D[:, dV].  Warp 2 brings Q and the
-//     chunk's K, [V, 1]^T blocks by TMA.
+//   tc_readout       one CTA (512 threads) per (head, 256 tokens = two
+//     128-token blocks of one chunk), launched heaviest first (later chunks
+//     first, chunk 0 last): D_b[128 x NP] in TMEM accumulates phi(Q_b) S_(c-1)
+//     over the tiles of 64 basis rows (warps 8-15, one thread per token = TMEM
+//     lane, generate the tiles' monomials into TMEM A stages; warp 0 streams
+//     the snapshot tiles by TMA, each feeding both blocks) plus the in-chunk
+//     part sum_{c0 <= j <= i} T_4(s_ij) [v_j, 1] per 64-key block: scores
+//     Q K^T into TMEM, T_4 and the causal mask by the epilogue warps 4-7, P
+//     split into bf16 hi + lo parts (T_4 rounded to bf16 loses too much on
+//     rows whose denominator cancels), P_hi [V, 1] + P_lo [V, 1] into D_b;
+//     out = D[:, :dV] / D[:, dV].  Warp 2 brings Q and the chunk's K,
+//     [V, 1]^T blocks by TMA; warps 1 and 3 (one thread each) issue block 0's
+//     and block 1's MMAs.
 //
 // An MMA-issuing thread waits on one barrier per stage: a wait there stalls
 // the tensor pipe, whose queue holds only a couple of MMAs.  Every mbarrier
@@ -563,10 +565,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + S::ROffBar);
   uint64_t *q_full = bar, *kv_full = bar + 1, *kv_empty = bar + 2, *s_full = bar + 3,
            *p_full = bar + 4, *o_full = bar + 5, *a_full = bar + 6, *a_empty = a_full + kRStages,
-           *b_full = a_empty + kRStages, *b_empty = b_full + kRBS;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(b_empty + kRBS);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(b_empty + kRBS + 1);
-  static_assert((6 + 2 * kRStages + 2 * kRBS + 2) * 8 <= 512, "barrier region");
+           *b_full = a_empty + kRStages, *b_empty = b_full + kRBS, *blk0_done = b_empty + kRBS;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(blk0_done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(blk0_done + 2);
+  static_assert((7 + 2 * kRStages + 2 * kRBS + 2) * 8 <= 512, "barrier region");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // heaviest first: the last pairs of blocks (in the last chunks, with the
@@ -591,15 +593,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(kv_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(p_full, 4);
-    mbar_init(o_full, 1);
+    mbar_init(o_full, 2);  // one commit per MMA issuer
     for (int s = 0; s < kRStages; ++s) {
       mbar_init(&a_full[s], 8);
-      mbar_init(&a_empty[s], 1);
+      mbar_init(&a_empty[s], 2);
     }
     for (int s = 0; s < kRBS; ++s) {
       mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], 1);
+      mbar_init(&b_empty[s], 2);
     }
+    mbar_init(blk0_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -655,19 +658,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(q_full, 0, &never, p.err);
       if (jb > 0) mbar_wait(kv_full, (jb - 1) & 1, &never, p.err);
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ---------------- MMA issuers: warp 1 issues every MMA of block 0, warp 3
+    // every MMA of block 1 (one thread issues an MMA only every ~60-80
+    // cycles, an M = 128, N = NP MMA takes NP / 2), so no accumulator is
+    // written from two threads
     if (lane == 0) {
+      const int b = warp == 1 ? 0 : 1;
       constexpr uint32_t id_nv = idesc_bf16_f32(128, NP, false, false);  // B: NP rows, K-major
       constexpr uint32_t id_qk = idesc_bf16_f32(128, kKB, false, false);
-      bool d_init[2] = {false, false}, ok = true;
-      int jq = 0, jp = 0;  // next job for scores / for P [V, 1]
-      const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), vt0 = smem_u32(sVT);
+      const uint32_t d_blk = tmem + b * NP;
+      bool d_init = false, ok = true;
+      // this block's in-chunk jobs: [j0, j1) of the CTA's job list (block 0's
+      // first; the K / V block, score and P buffers pass from job to job
+      // through kv_empty, whatever thread issued the previous job)
+      const int j0 = b == 0 ? 0 : nkb0, j1 = b == 0 ? nkb0 : njobs;
+      int jq = j0, jp = j0;  // next job for scores / for P [V, 1]
+      const uint32_t q0 = smem_u32(sQ) + b * kRTile, k0 = smem_u32(sK), vt0 = smem_u32(sVT);
       const uint32_t p0 = smem_u32(sP);
       ok = mbar_wait(q_full, 0, abort_flag, p.err, p.wait_limit);
+      // block 1's jobs start once block 0's are complete (before that its
+      // barriers may lag by more than the one phase a parity wait can tell)
+      bool jobs_open = b == 0;
       // in-chunk part, advanced whenever its inputs are ready
       auto intra = [&](bool block) {
-        while (ok && jp < njobs) {
+        if (ok && !jobs_open && jp < j1) {
+          if (block) {
+            if (!(ok = mbar_wait(blk0_done, 0, abort_flag, p.err, p.wait_limit))) return;
+          } else if (!mbar_test_wait(blk0_done, 0)) {
+            return;
+          }
+          jobs_open = true;
+        }
+        while (ok && jp < j1) {
           if (jq == jp) {  // next: scores of job jq
             if (block) {
               if (!(ok = mbar_wait(kv_full, jq & 1, abort_flag, p.err, p.wait_limit))) return;
@@ -675,32 +698,31 @@ __global__ void __launch_bounds__(kThreads, 1)
               return;
             }
             tc_fence_after();
-            const uint32_t qb = q0 + (jq < nkb0 ? 0u : kRTile);
 #pragma unroll
             for (int k = 0; k < DK / 16; ++k)
-              mma_bf16_ss(tS, smem_desc_sw128(qb + 32 * k, 16, 1024),
+              mma_bf16_ss(tS, smem_desc_sw128(q0 + 32 * k, 16, 1024),
                           smem_desc_sw128(k0 + 32 * k, 16, 1024), id_qk, k > 0 ? 1u : 0u);
             mma_commit(s_full);
             ++jq;
-          } else {  // next: P [V, 1] of job jp into its block's accumulator
+          } else {  // next: P [V, 1] of job jp into the block's accumulator
             if (block) {
               if (!(ok = mbar_wait(p_full, jp & 1, abort_flag, p.err, p.wait_limit))) return;
             } else if (!mbar_test_wait(p_full, jp & 1)) {
               return;
             }
             tc_fence_after();
-            const int b = jp < nkb0 ? 0 : 1;
 #pragma unroll
             for (int k = 0; k < 2 * (kKB / 16); ++k) {  // hi part, then lo part
               const int kk = k % (kKB / 16);
               const uint64_t ad =
                   smem_desc_sw128(p0 + (k / (kKB / 16)) * kRTile + 32 * kk, 16, 1024);
               const uint64_t bd = smem_desc_sw128(vt0 + 32 * kk, 16, 1024);
-              mma_bf16_ss(tmem + b * NP, ad, bd, id_nv, (d_init[b] || k > 0) ? 1u : 0u);
+              mma_bf16_ss(d_blk, ad, bd, id_nv, (d_init || k > 0) ? 1u : 0u);
             }
-            d_init[b] = true;
+            d_init = true;
             mma_commit(kv_empty);
             ++jp;
+            if (b == 0 && jp == j1) mma_commit(blk0_done);
           }
         }
       };
@@ -716,20 +738,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           tc_fence_after();
           const int nt = min(kRTS, p.n_tiles - kRTS * i);
-          // each block's MMAs back to back on its own accumulator (MMAs that
-          // switch accumulators run several times slower); both read the
-          // stage's snapshot tiles
+          for (int t = 0; t < nt; ++t) {
+            const uint64_t bd = smem_desc_sw128(b0 + (bs * kRTS + t) * S::RB, 16, 1024);
+            const uint32_t ad = tmem + ColA + ((st * 2 + b) * kRTS + t) * 32;
 #pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            for (int t = 0; t < nt; ++t) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16_ts(tmem + b * NP, tmem + ColA + ((st * 2 + b) * kRTS + t) * 32 + 8 * k,
-                            smem_desc_sw128(b0 + (bs * kRTS + t) * S::RB + 32 * k, 16, 1024),
-                            id_nv, (d_init[b] || t > 0 || k > 0) ? 1u : 0u);
-            }
+            for (int k = 0; k < 4; ++k)
+              mma_bf16_ts(d_blk, ad + 8 * k, bd + 2 * k, id_nv, (d_init || t > 0 || k > 0) ? 1u : 0u);
           }
-          d_init[0] = d_init[1] = true;
+          d_init = true;
           mma_commit(&a_empty[st]);
           mma_commit(&b_empty[bs]);
           intra(false);
