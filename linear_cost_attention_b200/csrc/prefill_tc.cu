@@ -81,7 +81,8 @@ constexpr int kChunk = 4096;     // tokens per chunk (a multiple of the 128-toke
 // ------------------------------------------------------------ readout
 constexpr int kThreads = 512;
 constexpr int kMaxTiles = 768;           // tile table capacity in smem
-constexpr int kRTS = 2;                  // feature tiles per pipeline stage
+constexpr int kRTS = 2;                  // feature tiles per pipeline stage (the generators
+                                         // take consecutive OUTER tiles in pairs)
 constexpr int kRStages = 2;              // phi(Q) stages, in TMEM (2 blocks x 32 columns per tile)
 constexpr int kRBS = 4;                  // snapshot stages (kRTS tiles each)
 constexpr int kKB = 64;                  // keys per in-chunk block
@@ -833,20 +834,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i >= kRStages && !(ok = mbar_wait(&a_empty[st], ((i / kRStages) - 1) & 1, abort_flag,
                                             p.err, p.wait_limit)))
         break;
+      // this thread's token is TMEM lane `row` of block b; a tile's 64
+      // features are 32 packed columns
+      const uint32_t acol = tmem + tl + ColA + (st * 2 + b) * kRTS * 32;
+      const TileDesc pad{T_PAD, 0, 0, 0, 0, 0, 0, 0};
+      const TileDesc d0 = kRTS * i < p.n_tiles ? sTiles[kRTS * i] : pad;
+      const TileDesc d1 = kRTS * i + 1 < p.n_tiles ? sTiles[kRTS * i + 1] : pad;
+      if (outer_pair_ok(d0, d1)) {
+        // the stage's two tiles share their octets (most OUTER tiles)
+        uint32_t out0[32], out1[32];
+        gen_outer_pair(d0, qrow, (uint32_t)(row & 7), p.W, out0, out1);
+        tmem_st32(acol, out0);
+        tmem_st32(acol + 32, out1);
+      } else {
 #pragma unroll 1
-      for (int t = 0; t < kRTS; ++t) {
-        const int ti = kRTS * i + t;
-        uint32_t out[32];
-        if (ti < p.n_tiles) {
-          const TileDesc td = sTiles[ti];
-          gen_tile<S::G>(td, qrow, (uint32_t)(row & 7), p.W, out);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 32; ++q) out[q] = 0u;
+        for (int t = 0; t < kRTS; ++t) {
+          uint32_t out[32];
+          gen_tile<S::G>(t ? d1 : d0, qrow, (uint32_t)(row & 7), p.W, out);
+          tmem_st32(acol + 32 * t, out);
         }
-        // this thread's token is TMEM lane `row` of block b; a tile's 64
-        // features are 32 packed columns
-        tmem_st32(tmem + tl + ColA + ((st * 2 + b) * kRTS + t) * 32, out);
       }
       tmem_st_wait();
       if (!(ok = mbar_wait(&b_full[i % kRBS], (i / kRBS) & 1, abort_flag, p.err, p.wait_limit)))

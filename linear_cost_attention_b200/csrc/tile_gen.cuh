@@ -7,11 +7,13 @@
 // 0..3 are read.  The 64 outputs are returned as 32 packed bf16x2 words in
 // tile order.
 //
-// Arithmetic (feature = w_alpha * prod x): OUTER and BC tiles form the pair
-// product u = w * x_i * x_j in fp32, round it to bf16 and multiply by the
-// eight values of the third octet with packed bf16x2 multiplies (two
-// roundings); D and MISC tiles (21 of 749) load the octets they touch once and
-// form each product in fp32, rounding once.
+// Arithmetic (feature = w_alpha * prod x): OUTER and BC tiles form bf16x2
+// pairs of partial products u = w * x_i * x_j (OUTER: w x_i rounded to bf16,
+// exact for the unit weights the readout uses, times x_j with a packed
+// multiply; BC: in fp32) rounded to bf16, and multiply them by the packed
+// words of the third octet, halves swapped or not (two roundings); D and MISC
+// tiles (21 of 749) load the octets they touch once and form each product in
+// fp32, rounding once.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -95,48 +97,81 @@ SATA_HD uint32_t pack2(float lo, float hi) {
 }
 
 // u * (8 values of chunk r) -> out[4*slot .. 4*slot+3]
-SATA_HD void scale_chunk(float u, uint4 r, uint32_t *out4) {
-  const uint32_t uu = splat_bf16(u);
-  out4[0] = bmul2(uu, r.x);
-  out4[1] = bmul2(uu, r.y);
-  out4[2] = bmul2(uu, r.z);
-  out4[3] = bmul2(uu, r.w);
+// 32-bit word holding elements i and i + 1 (i even) of the row.
+SATA_HD uint32_t load_pair(const uint8_t *row, uint32_t rsw, int i) {
+  return *reinterpret_cast<const uint32_t *>(row + ((((uint32_t)i >> 3) ^ rsw) << 4) +
+                                             ((i & 7) << 1));
 }
 
-SATA_HD void gen_outer(const TileDesc &td, const uint8_t *row, uint32_t rsw,
-                                          const GenWeights &W, uint32_t (&out)[32]) {
-  float ob[8];
-  unpack8(load_chunk(row, rsw, td.o0), ob);
-  const uint4 rc = load_chunk(row, rsw, td.o1);
-  const float s =
-      (td.wsel == 0 ? W.w3 : W.w2) * (td.i1 != kNoIndex ? load_elem(row, rsw, td.i1) : 1.f);
+SATA_HD uint32_t swap_halves(uint32_t x) { return (x >> 16) | (x << 16); }
+
+// The 32 words of an OUTER / BC tile from four bf16x2 pairs of partial
+// products u[k] (word w uses u[w / 8]) and the third octet's chunk r: word w
+// = u[w / 8] * r_j or * swap(r_j), j = (w % 8) / 2 (tile_order.h, outer_c).
+SATA_HD void outer_words(const uint32_t (&u)[4], uint4 r, uint32_t (&out)[32]) {
+  const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-  for (int b = 0; b < 8; ++b) scale_chunk(s * ob[b], rc, &out[4 * b]);
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t rs = swap_halves(rw[j]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      out[8 * k + 2 * j] = bmul2(u[k], rw[j]);
+      out[8 * k + 2 * j + 1] = bmul2(u[k], rs);
+    }
+  }
 }
 
-// ---- BC: chunk CC of variant T
+// OUTER: u pairs (s x_b, s x_(b+1)) with s = w x_i1 (w alone for degree 2),
+// rounded to bf16, times the third octet's words.
+SATA_HD void gen_outer(const TileDesc &td, const uint8_t *row, uint32_t rsw,
+                       const GenWeights &W, uint32_t (&out)[32]) {
+  const uint4 g = load_chunk(row, rsw, td.o0);
+  const uint4 rc = load_chunk(row, rsw, td.o1);
+  const uint32_t sp = splat_bf16(
+      (td.wsel == 0 ? W.w3 : W.w2) * (td.i1 != kNoIndex ? load_elem(row, rsw, td.i1) : 1.f));
+  const uint32_t u[4] = {bmul2(sp, g.x), bmul2(sp, g.y), bmul2(sp, g.z), bmul2(sp, g.w)};
+  outer_words(u, rc, out);
+}
+
+// Two consecutive degree-3 OUTER tiles that differ only in i1 (i1 even, then
+// i1 + 1): the octet chunks and the i1 pair are loaded once.
+SATA_HD void gen_outer_pair(const TileDesc &td, const uint8_t *row, uint32_t rsw,
+                            const GenWeights &W, uint32_t (&out0)[32], uint32_t (&out1)[32]) {
+  const uint4 g = load_chunk(row, rsw, td.o0);
+  const uint4 rc = load_chunk(row, rsw, td.o1);
+  const uint32_t xi = load_pair(row, rsw, td.i1);
+  const uint32_t s0 = splat_bf16(W.w3 * bf16_bits_to_f32(xi & 0xffffu));
+  const uint32_t s1 = splat_bf16(W.w3 * bits_f32(xi & 0xffff0000u));
+  const uint32_t u0[4] = {bmul2(s0, g.x), bmul2(s0, g.y), bmul2(s0, g.z), bmul2(s0, g.w)};
+  const uint32_t u1[4] = {bmul2(s1, g.x), bmul2(s1, g.y), bmul2(s1, g.z), bmul2(s1, g.w)};
+  outer_words(u0, rc, out0);
+  outer_words(u1, rc, out1);
+}
+
+// True when tiles t, t + 1 can take gen_outer_pair.
+SATA_HD bool outer_pair_ok(const TileDesc &a, const TileDesc &b) {
+  return a.type == T_OUTER && b.type == T_OUTER && a.i1 != kNoIndex && (a.i1 & 1) == 0 &&
+         b.i1 == a.i1 + 1 && a.o0 == b.o0 && a.o1 == b.o1 && a.wsel == b.wsel;
+}
+
+// ---- BC: tile variant T; chunk cc holds pair k = 8 T + cc (block k / 36 of
+// the tile's two octet pairs); chunks 2q, 2q + 1 share the third octet
 template <int T, int CC>
-SATA_HD void bc_chunk(const float (&g0)[8], uint4 r0, const float (&g1)[8],
-                                         uint4 r1, const GenWeights &W, uint32_t (&out)[32]) {
+SATA_HD float bc_pair_product(const float (&g0)[8], const float (&g1)[8], const GenWeights &W) {
   constexpr int k = 8 * T + CC, blk = k / 36, p = k % 36;
   constexpr int a = pair_a(p), b = pair_b(p);
   const float w = (a == b) ? W.w3h : W.w3;
-  if (blk == 0)
-    scale_chunk(w * g0[a] * g0[b], r0, &out[4 * CC]);
-  else
-    scale_chunk(w * g1[a] * g1[b], r1, &out[4 * CC]);
+  return blk == 0 ? w * g0[a] * g0[b] : w * g1[a] * g1[b];
 }
 
-template <int T, int... CC>
-SATA_HD void bc_variant(const float (&g0)[8], uint4 r0, const float (&g1)[8],
-                                           uint4 r1, const GenWeights &W, uint32_t (&out)[32],
-                                           std::integer_sequence<int, CC...>) {
-  (bc_chunk<T, CC>(g0, r0, g1, r1, W, out), ...);
+template <int T, int Q>
+SATA_HD uint32_t bc_u(const float (&g0)[8], const float (&g1)[8], const GenWeights &W) {
+  return pack2(bc_pair_product<T, 2 * Q>(g0, g1, W), bc_pair_product<T, 2 * Q + 1>(g0, g1, W));
 }
 
 template <int T>
 SATA_HD void gen_bc(const TileDesc &td, const uint8_t *row, uint32_t rsw,
-                                       const GenWeights &W, uint32_t (&out)[32]) {
+                    const GenWeights &W, uint32_t (&out)[32]) {
   constexpr bool need0 = 8 * T < 36, need1 = 8 * T + 7 >= 36;
   float g0[8] = {0, 0, 0, 0, 0, 0, 0, 0}, g1[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
@@ -148,7 +183,21 @@ SATA_HD void gen_bc(const TileDesc &td, const uint8_t *row, uint32_t rsw,
     unpack8(load_chunk(row, rsw, td.o2), g1);
     r1 = load_chunk(row, rsw, td.o3);
   }
-  bc_variant<T>(g0, r0, g1, r1, W, out, std::make_integer_sequence<int, 8>{});
+  const uint32_t u[4] = {bc_u<T, 0>(g0, g1, W), bc_u<T, 1>(g0, g1, W), bc_u<T, 2>(g0, g1, W),
+                         bc_u<T, 3>(g0, g1, W)};
+  // the block boundary (pair 36) falls on an even chunk, so both chunks of a
+  // word use one third octet; words of chunks in block 1 use r1
+  const uint32_t rw0[4] = {r0.x, r0.y, r0.z, r0.w}, rw1[4] = {r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const bool b1 = (8 * T + 2 * q) >= 36;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t rj = b1 ? rw1[j] : rw0[j];
+      out[8 * q + 2 * j] = bmul2(u[q], rj);
+      out[8 * q + 2 * j + 1] = bmul2(u[q], swap_halves(rj));
+    }
+  }
 }
 
 // ---- D: features 64*T + P of the concatenated in-octet triples; a tile

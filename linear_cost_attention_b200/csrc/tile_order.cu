@@ -52,8 +52,11 @@ bool build_tile_order(int dK, TileOrder *out) {
     for (int gj = gi + 1; gj < G; ++gj)
       for (int gl = gj + 1; gl < G; ++gl)
         for (int a = 0; a < 8; ++a) {
-          for (int b = 0; b < 8; ++b)
-            for (int c = 0; c < 8; ++c) s[8 * b + c] = sorted3(8 * gi + a, 8 * gj + b, 8 * gl + c);
+          for (int w = 0; w < 32; ++w) {
+            const int b = outer_b(w), c0 = outer_c(w, 0), c1 = outer_c(w, 1);
+            s[2 * w] = sorted3(8 * gi + a, 8 * gj + b, 8 * gl + c0);
+            s[2 * w + 1] = sorted3(8 * gi + a, 8 * gj + b + 1, 8 * gl + c1);
+          }
           push({T_OUTER, 0, (uint8_t)(8 * gi + a), (uint8_t)gj, (uint8_t)gl, 0, 0, 0}, s);
         }
   // BC: pairs of ordered octet pairs (g, g'), g != g'
@@ -64,12 +67,14 @@ bool build_tile_order(int dK, TileOrder *out) {
   for (size_t bp = 0; bp + 1 < og.size(); bp += 2) {
     const auto b0 = og[bp], b1 = og[bp + 1];
     for (int t = 0; t < 9; ++t) {
-      for (int cc = 0; cc < 8; ++cc) {
-        const int k = 8 * t + cc, blk = k / 36, p = k % 36;
-        const int a = pair_a(p), b = pair_b(p);
-        const auto gg = blk ? b1 : b0;
-        for (int e = 0; e < 8; ++e)
-          s[8 * cc + e] = sorted3(8 * gg.first + a, 8 * gg.first + b, 8 * gg.second + e);
+      for (int w = 0; w < 32; ++w) {
+        // word w: chunks cc, cc + 1 (one pair each) times the third octet
+        for (int h = 0; h < 2; ++h) {
+          const int cc = 2 * (w / 8) + h, k = 8 * t + cc, blk = k / 36, p = k % 36;
+          const int a = pair_a(p), b = pair_b(p);
+          const auto gg = blk ? b1 : b0;
+          s[2 * w + h] = sorted3(8 * gg.first + a, 8 * gg.first + b, 8 * gg.second + outer_c(w, h));
+        }
       }
       push({T_BC, (uint8_t)t, 0, (uint8_t)b0.first, (uint8_t)b0.second, (uint8_t)b1.first,
             (uint8_t)b1.second, 0},
@@ -79,8 +84,10 @@ bool build_tile_order(int dK, TileOrder *out) {
   // OUTER, degree 2: two distinct octets
   for (int g = 0; g < G; ++g)
     for (int h = g + 1; h < G; ++h) {
-      for (int b = 0; b < 8; ++b)
-        for (int c = 0; c < 8; ++c) s[8 * b + c] = sorted2(8 * g + b, 8 * h + c);
+      for (int w = 0; w < 32; ++w) {
+        s[2 * w] = sorted2(8 * g + outer_b(w), 8 * h + outer_c(w, 0));
+        s[2 * w + 1] = sorted2(8 * g + outer_b(w) + 1, 8 * h + outer_c(w, 1));
+      }
       push({T_OUTER, 0, kNoIndex, (uint8_t)g, (uint8_t)h, 0, 0, 1}, s);
     }
   // D: triples inside one octet

@@ -65,6 +65,17 @@ __host__ __device__ constexpr int triple_at(int r, int which) {
       }
   return 0;
 }
+// Feature order inside OUTER and BC tiles.  Packed word w (features 2w, 2w+1)
+// holds two products with the third octet's entries c0 = outer_c(w, 0),
+// c1 = outer_c(w, 1), which are (2j, 2j+1) or (2j+1, 2j) for j = (w % 8) / 2:
+// the generator multiplies a bf16x2 pair of partial products by one packed
+// word of the third octet or by that word with its halves swapped.  OUTER:
+// partial products for b = outer_b(w) and b + 1 of the first octet; BC: the
+// pairs of chunks 2 (w / 8) and 2 (w / 8) + 1.
+__host__ __device__ constexpr int outer_b(int w) { return 2 * (w / 8); }
+__host__ __device__ constexpr int outer_c(int w, int half) {
+  return 2 * ((w % 8) / 2) + ((w % 2) ^ half);
+}
 // alpha! of a sorted triple / pair with equal-index runs
 __host__ __device__ constexpr int fact3(int a, int b, int c) {
   return (a == b && b == c) ? 6 : (a == b || b == c) ? 2 : 1;

@@ -20,8 +20,11 @@
 
 using namespace sata;
 
+// unit_weights: the readout's configuration (unweighted monomials; the
+// weights live in the snapshots); then every feature is at most two bf16
+// roundings from the exact product, else three (the weight adds one).
 template <int G>
-int check(int dK, int want_tiles) {
+int check(int dK, int want_tiles, bool unit_weights) {
   TileOrder to;
   if (!build_tile_order(dK, &to)) {
     printf("FAIL build_tile_order dK=%d\n", dK);
@@ -43,6 +46,9 @@ int check(int dK, int want_tiles) {
   W.w2 = (float)(1.0 / std::sqrt(d));
   W.w2h = (float)(1.0 / std::sqrt(2.0 * d));
   W.w1 = (float)(1.0 / std::sqrt(std::sqrt(d)));
+  if (unit_weights) W = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+  const double u = std::ldexp(1.0, -8);  // bf16 unit roundoff
+  const double bound = unit_weights ? (1 + u) * (1 + u) - 1 : (1 + u) * (1 + u) * (1 + u) - 1;
   std::mt19937 rng(1234 + dK);
   std::normal_distribution<float> nd(0.f, 1.f);
   double worst = 0;
@@ -75,11 +81,11 @@ int check(int dK, int want_tiles) {
         const int32_t row_id = to.row_of_slot[(size_t)t * 64 + p];
         double ref = 0.0;
         if (row_id >= 0) {
-          ref = hb.weight[row_id];
+          ref = unit_weights ? 1.0 : hb.weight[row_id];
           for (int s = 0; s < hb.degree[row_id]; ++s) ref *= x[hb.ix[4 * row_id + s]];
         }
         const double err = std::fabs(got - ref);
-        const double tol = 3 * std::ldexp(1.0, -8) * std::fabs(ref) + 1e-30;
+        const double tol = bound * std::fabs(ref) + 1e-30;
         if (row_id < 0 ? got != 0.f : err > tol) {
           if (bad < 10)
             printf("mismatch dK %d tile %d type %d var %d slot %d row %d got %g ref %g\n", dK, t,
@@ -90,7 +96,28 @@ int check(int dK, int want_tiles) {
       }
     }
   }
-  printf("dK %d: worst relative %.3e bad %ld\n", dK, worst, bad);
+  // the readout's two-tile path equals the one-tile path bit for bit
+  long pair_bad = 0, pairs = 0;
+  for (int trial = 0; trial < 4; ++trial) {
+    const uint32_t r = trial % 8;
+    alignas(16) uint8_t row[128];
+    for (int i = 0; i < 128; i += 2) {
+      __nv_bfloat16 b = __float2bfloat16_rn(nd(rng));
+      memcpy(row + i, &b, 2);
+    }
+    for (int t = 0; t + 1 < to.n_tiles; ++t) {
+      if (!tc::outer_pair_ok(to.tiles[t], to.tiles[t + 1])) continue;
+      ++pairs;
+      uint32_t a0[32], a1[32], b0[32], b1[32];
+      tc::gen_tile<G>(to.tiles[t], row, r, W, a0);
+      tc::gen_tile<G>(to.tiles[t + 1], row, r, W, a1);
+      tc::gen_outer_pair(to.tiles[t], row, r, W, b0, b1);
+      pair_bad += memcmp(a0, b0, sizeof a0) != 0 || memcmp(a1, b1, sizeof a1) != 0;
+    }
+  }
+  bad += pair_bad;
+  printf("dK %d%s: worst relative %.3e (bound %.3e) bad %ld, %ld two-tile checks\n", dK,
+         unit_weights ? " unit weights" : "", worst, bound, bad, pairs);
   return bad ? 1 : 0;
 }
 
@@ -164,7 +191,8 @@ int check_groups(int dK) {
 }
 
 int main() {
-  int fails = check<8>(64, 749) + check<4>(32, 103) + check_groups(64) + check_groups(32);
+  int fails = check<8>(64, 749, false) + check<4>(32, 103, false) + check<8>(64, 749, true) +
+              check<4>(32, 103, true) + check_groups(64) + check_groups(32);
   if (fails) {
     printf("FAIL\n");
     return 1;
