@@ -543,6 +543,81 @@ struct RParams {
   long long wait_limit;  // cycles before a role's wait gives up (drains: full limit)
 };
 
+// Generates one tile for this thread's token and stores it to TMEM at taddr
+// (32 columns).  Each case stores its own registers: a switch whose cases
+// only fill a shared output array makes the compiler merge the 32 outputs of
+// every case at the join, which costs more than the generation.
+template <int G>
+__device__ __forceinline__ void gen_store_tile(const TileDesc &td, const uint8_t *row,
+                                               uint32_t rsw, const GenWeights &W,
+                                               uint32_t taddr) {
+  uint32_t out[32];
+  switch (td.type) {
+    case T_OUTER: gen_outer(td, row, rsw, W, out); tmem_st32(taddr, out); return;
+    case T_BC:
+      switch (td.variant) {
+        case 0: gen_bc<0>(td, row, rsw, W, out); tmem_st32(taddr, out); return;
+        case 1: gen_bc<1>(td, row, rsw, W, out); tmem_st32(taddr, out); return;
+        case 2: gen_bc<2>(td, row, rsw, W, out); tmem_st32(taddr, out); return;
+        case 3: gen_bc<3>(td, row, rsw, W, out); tmem_st32(taddr, out); return;
+        case 4: gen_bc<4>(td, row, rsw, W, out); tmem_st32(taddr, out); return;
+        case 5: gen_bc<5>(td, row, rsw, W, out); tmem_st32(taddr, out); return;
+        case 6: gen_bc<6>(td, row, rsw, W, out); tmem_st32(taddr, out); return;
+        case 7: gen_bc<7>(td, row, rsw, W, out); tmem_st32(taddr, out); return;
+        default: gen_bc<8>(td, row, rsw, W, out); tmem_st32(taddr, out); return;
+      }
+    case T_D: gen_d<G>(td.variant, row, rsw, W, out); tmem_st32(taddr, out); return;
+    case T_MISC: gen_misc<G>(td.variant, row, rsw, W, out); tmem_st32(taddr, out); return;
+    default:
+#pragma unroll
+      for (int i = 0; i < 32; ++i) out[i] = 0u;
+      tmem_st32(taddr, out);
+      return;
+  }
+}
+
+template <int G, int T>
+__device__ __forceinline__ void gen_store_bc2(const TileDesc &d0, const TileDesc &d1,
+                                              const uint8_t *row, uint32_t rsw,
+                                              const GenWeights &W, uint32_t taddr) {
+  uint32_t out0[32], out1[32];
+  gen_bc<T>(d0, row, rsw, W, out0);
+  gen_bc<T>(d1, row, rsw, W, out1);
+  tmem_st32(taddr, out0);
+  tmem_st32(taddr + 32, out1);
+}
+
+// A stage's two tiles (tile order, tile_order.h): the tile order holds long
+// runs of one kind, so the stage dispatches once to straight-line code for
+// an OUTER pair or two BC tiles of one variant, else tile by tile.
+template <int G>
+__device__ __forceinline__ void gen_store_stage(const TileDesc &d0, const TileDesc &d1,
+                                                const uint8_t *row, uint32_t rsw,
+                                                const GenWeights &W, uint32_t taddr) {
+  if (outer_pair_ok(d0, d1)) {
+    uint32_t out0[32], out1[32];
+    gen_outer_pair(d0, row, rsw, W, out0, out1);
+    tmem_st32(taddr, out0);
+    tmem_st32(taddr + 32, out1);
+    return;
+  }
+  if (d0.type == T_BC && d1.type == T_BC && d0.variant == d1.variant) {
+    switch (d0.variant) {
+      case 0: gen_store_bc2<G, 0>(d0, d1, row, rsw, W, taddr); return;
+      case 1: gen_store_bc2<G, 1>(d0, d1, row, rsw, W, taddr); return;
+      case 2: gen_store_bc2<G, 2>(d0, d1, row, rsw, W, taddr); return;
+      case 3: gen_store_bc2<G, 3>(d0, d1, row, rsw, W, taddr); return;
+      case 4: gen_store_bc2<G, 4>(d0, d1, row, rsw, W, taddr); return;
+      case 5: gen_store_bc2<G, 5>(d0, d1, row, rsw, W, taddr); return;
+      case 6: gen_store_bc2<G, 6>(d0, d1, row, rsw, W, taddr); return;
+      case 7: gen_store_bc2<G, 7>(d0, d1, row, rsw, W, taddr); return;
+      default: gen_store_bc2<G, 8>(d0, d1, row, rsw, W, taddr); return;
+    }
+  }
+#pragma unroll 1
+  for (int t = 0; t < 2; ++t) gen_store_tile<G>(t ? d1 : d0, row, rsw, W, taddr + 32 * t);
+}
+
 __device__ __forceinline__ float taylor4(float s) {
   return fmaf(fmaf(fmaf(s, 1.0f / 6.0f, 0.5f), s, 1.0f), s, 1.0f);
 }
@@ -840,20 +915,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileDesc pad{T_PAD, 0, 0, 0, 0, 0, 0, 0};
       const TileDesc d0 = kRTS * i < p.n_tiles ? sTiles[kRTS * i] : pad;
       const TileDesc d1 = kRTS * i + 1 < p.n_tiles ? sTiles[kRTS * i + 1] : pad;
-      if (outer_pair_ok(d0, d1)) {
-        // the stage's two tiles share their octets (most OUTER tiles)
-        uint32_t out0[32], out1[32];
-        gen_outer_pair(d0, qrow, (uint32_t)(row & 7), p.W, out0, out1);
-        tmem_st32(acol, out0);
-        tmem_st32(acol + 32, out1);
-      } else {
-#pragma unroll 1
-        for (int t = 0; t < kRTS; ++t) {
-          uint32_t out[32];
-          gen_tile<S::G>(t ? d1 : d0, qrow, (uint32_t)(row & 7), p.W, out);
-          tmem_st32(acol + 32 * t, out);
-        }
-      }
+      static_assert(kRTS == 2, "stages of two tiles");
+      gen_store_stage<S::G>(d0, d1, qrow, (uint32_t)(row & 7), p.W, acol);
       tmem_st_wait();
       if (!(ok = mbar_wait(&b_full[i % kRBS], (i / kRBS) & 1, abort_flag, p.err, p.wait_limit)))
         break;

@@ -64,9 +64,10 @@ bool build_tile_order(int dK, TileOrder *out) {
   for (int g = 0; g < G; ++g)
     for (int h = 0; h < G; ++h)
       if (h != g) og.push_back({g, h});
-  for (size_t bp = 0; bp + 1 < og.size(); bp += 2) {
-    const auto b0 = og[bp], b1 = og[bp + 1];
-    for (int t = 0; t < 9; ++t) {
+  // variant-major: runs of tiles of one variant take one code path in a row
+  for (int t = 0; t < 9; ++t)
+    for (size_t bp = 0; bp + 1 < og.size(); bp += 2) {
+      const auto b0 = og[bp], b1 = og[bp + 1];
       for (int w = 0; w < 32; ++w) {
         // word w: chunks cc, cc + 1 (one pair each) times the third octet
         for (int h = 0; h < 2; ++h) {
@@ -80,7 +81,6 @@ bool build_tile_order(int dK, TileOrder *out) {
             (uint8_t)b1.second, 0},
            s);
     }
-  }
   // OUTER, degree 2: two distinct octets
   for (int g = 0; g < G; ++g)
     for (int h = g + 1; h < G; ++h) {

@@ -31,7 +31,7 @@ namespace sata {
 
 enum TileType : uint8_t { T_OUTER = 0, T_BC = 1, T_D = 2, T_MISC = 3, T_PAD = 4 };
 
-struct TileDesc {  // 8 bytes; read by the generator warps
+struct alignas(8) TileDesc {  // 8 bytes, one 64-bit load; read by the generator warps
   uint8_t type, variant, i1, o0, o1, o2, o3, wsel;
 };
 constexpr uint8_t kNoIndex = 0xff;  // OUTER tile of degree 2: no first index
