@@ -76,7 +76,10 @@ constexpr int kUMmaWarp1 = kUGenWarp0 + kUGenWarps;  // second MMA issuer (the f
 constexpr int kUThreads = 32 * (kUMmaWarp1 + 1);
 constexpr uint32_t kUTmemCols = 512;
 constexpr int kMaxDevices = 64;  // per-device launch attributes
-constexpr int kChunk = 4096;     // tokens per chunk (a multiple of the 128-token padding)
+// tokens per chunk (a multiple of the 256-token readout pairs): dK = 64 4096,
+// dK = 32 1024 (its state of 6545 rows makes the inter-chunk readout cheap
+// next to the in-chunk quadratic part, whose Taylor terms run on CUDA cores)
+template <int DK> constexpr int kChunk = DK == 64 ? 4096 : 1024;
 
 // ------------------------------------------------------------ readout
 constexpr int kThreads = 512;
@@ -978,9 +981,9 @@ int launch_tc(const void *q, const void *k, const void *v, float *out, float *st
   const int m_pad = n_tiles * 64;
   // Chunk length: a snapshot boundary stalls the state kernel while the tile
   // leaves TMEM and costs a snapshot write, while the readout hides the longer
-  // in-chunk quadratic part behind its inter-chunk MMAs; 4096 measured fastest
-  // of 1024 / 2048 / 4096 at 16384 tokens.
-  const int C = N <= kChunk ? ((N + 255) / 256) * 256 : kChunk;  // whole readout pairs
+  // in-chunk quadratic part behind its inter-chunk MMAs; at dK = 64 4096
+  // measured fastest of 1024 / 2048 / 4096 at 16384 tokens.
+  const int C = N <= kChunk<DK> ? ((N + 255) / 256) * 256 : kChunk<DK>;  // whole readout pairs
   // snapshots: the state before each chunk but the first, plus (continued
   // prefill) the initial state before chunk 0 in slot 0
   const int nsnap = (N + C - 1) / C - 1 + (cont ? 1 : 0);

@@ -154,9 +154,10 @@ def test_tensor_core_prefill_shapes(B, H, N):
 @pytest.mark.parametrize("B,H,N", [
     (1, 1, 1),        # one token
     (2, 3, 100),      # ragged, one partial key block
-    (1, 2, 4096),     # exactly one full chunk
-    (1, 1, 4224),     # one snapshot + a block of the next chunk
-    (2, 1, 9000),     # two snapshots, ragged tail
+    (1, 2, 1024),     # exactly one full chunk (1024 tokens at dK = 32)
+    (1, 1, 1280),     # one snapshot + a block of the next chunk
+    (1, 2, 4096),     # four chunks, three snapshots
+    (2, 1, 9000),     # eight snapshots, ragged tail
 ])
 def test_tensor_core_prefill_shapes_dk32(B, H, N):
     # bf16, dK = dV = 32, P = 4: the tcgen05 path with 4 index octets and N = 48
