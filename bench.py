@@ -496,7 +496,7 @@ def run_ours(args, rank, world, local_rank):
             "latency_flatness": max(quarters) / min(quarters) - 1.0,
             "roofline": {"bound": "hbm", "kernel": kname, "achieved": ach,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
-                         "traffic": traffic_record(kname),
+                         "traffic": traffic_record(kname if label == "fp32" else kname + ":mixed"),
                          "peak_source": pk["source"], "kernel_ms": kms,
                          "algorithmic_bytes_per_launch": dbytes},
         }
