@@ -153,142 +153,6 @@ struct LaneGroup {
   bool valid[kGroupRows];
 };
 
-// dK = 64: quarter-units of 32 lanes (one warp's TMEM lane quarter) whose
-// factors l = s and third[f] = t_f are the same in every lane, so that the
-// warp's loads of those rows are broadcasts, and whose own factors j come as
-// four whole index octets, one per 8-lane phase of the load, so that the only
-// per-lane load has no bank conflict.  Every monomial {a, b, c} of degree 3
-// over symbols 0..63 and ONE = 64 (the ones row) is assigned to exactly one
-// (s, t, j) split:
-//  * three distinct octets: each octet triple is given to one of its octet
-//    pairs (X, Y) so that every chosen pair holds four triples; quarter-unit =
-//    s in X, four t in Y, j over the pair's four third octets (224 units);
-//  * two or three indices in one octet A: the 36 index pairs of A are split
-//    into 9 stars of 4 pairs with a common index (the centre s); j runs over
-//    the other 7 octets and over A itself from the pair's larger index on
-//    (144 units, the lanes below it are padding);
-//  * degree 2 across octets {ONE, b, c}: s = ONE, four t in octet B, j over
-//    four octets given to B (14 units);
-//  * the rest (degree 2 inside an octet, degree 1, degree 0): lanes with
-//    s = ONE, j = c and up to four third factors each (4 units, not uniform).
-void groups_uniform64(std::vector<LaneGroup> &lg) {
-  const int ONES = 64;
-  auto quarter = [&](int sh, const int (&t)[4], const int (&oct)[4], auto valid) {
-    for (int k = 0; k < 4; ++k)
-      for (int r = 0; r < 8; ++r) {
-        LaneGroup g;
-        g.j = 8 * oct[k] + r;
-        g.l = sh;
-        for (int f = 0; f < kGroupRows; ++f) {
-          g.third[f] = t[f];
-          g.valid[f] = valid(f, g.j);
-        }
-        lg.push_back(g);
-      }
-  };
-  auto all = [](int, int) { return true; };
-  // (1) octet triples: the octets split into halves {0..3}, {4..7}; a triple
-  // with two octets in one half goes to that pair, except the offloads below
-  // (to the pairs (0,4), (1,5)); a triple inside a half goes to the listed pair
-  std::map<std::pair<int, int>, std::vector<int>> thirds;
-  auto give = [&](int x, int y, int c) { thirds[{std::min(x, y), std::max(x, y)}].push_back(c); };
-  const int inside[8][5] = {{0, 1, 2, 0, 1}, {0, 1, 3, 0, 3}, {0, 2, 3, 0, 2}, {1, 2, 3, 1, 2},
-                            {4, 5, 6, 4, 5}, {4, 5, 7, 4, 7}, {4, 6, 7, 4, 6}, {5, 6, 7, 5, 6}};
-  const int offload[8][5] = {{0, 1, 5, 1, 5}, {0, 3, 4, 0, 4}, {0, 2, 4, 0, 4}, {1, 2, 5, 1, 5},
-                             {4, 5, 1, 1, 5}, {4, 7, 0, 0, 4}, {4, 6, 0, 0, 4}, {5, 6, 1, 1, 5}};
-  for (int a = 0; a < 8; ++a)
-    for (int b = a + 1; b < 8; ++b)
-      for (int c = b + 1; c < 8; ++c) {
-        int e0 = -1, e1 = -1;
-        for (const auto &q : inside)
-          if (q[0] == a && q[1] == b && q[2] == c) e0 = q[3], e1 = q[4];
-        if (e0 < 0) {
-          // two octets of the triple share a half: that pair, unless offloaded
-          const int h[3] = {a / 4, b / 4, c / 4};
-          int x, y, z;
-          if (h[0] == h[1]) x = a, y = b, z = c;
-          else if (h[0] == h[2]) x = a, y = c, z = b;
-          else x = b, y = c, z = a;
-          e0 = x, e1 = y;
-          for (const auto &q : offload)
-            if (std::min(q[0], q[1]) == x && std::max(q[0], q[1]) == y && q[2] == z)
-              e0 = q[3], e1 = q[4];
-        }
-        const int c3 = a + b + c - e0 - e1;
-        give(e0, e1, c3);
-      }
-  for (const auto &kv : thirds) {
-    const int X = kv.first.first, Y = kv.first.second;
-    if (kv.second.size() != 4) {
-      lg.clear();
-      return;
-    }
-    const int oct[4] = {kv.second[0], kv.second[1], kv.second[2], kv.second[3]};
-    for (int x = 0; x < 8; ++x)
-      for (int h = 0; h < 2; ++h) {
-        const int t[4] = {8 * Y + 4 * h, 8 * Y + 4 * h + 1, 8 * Y + 4 * h + 2, 8 * Y + 4 * h + 3};
-        quarter(8 * X + x, t, oct, all);
-      }
-  }
-  // (2) stars of index pairs inside octet A (positions 0..7): position v < 7
-  // takes its own pair and the pairs with v-1, v-2, v-3 (mod 7); position 7
-  // takes its pairs in two stars
-  int stars[9][5];
-  for (int v = 0; v < 7; ++v) {
-    stars[v][0] = v;
-    stars[v][1] = v;
-    for (int d = 1; d <= 3; ++d) stars[v][1 + d] = (v - d + 7) % 7;
-  }
-  const int s7[2][4] = {{7, 0, 1, 2}, {3, 4, 5, 6}};
-  for (int k = 0; k < 2; ++k) {
-    stars[7 + k][0] = 7;
-    for (int f = 0; f < 4; ++f) stars[7 + k][1 + f] = s7[k][f];
-  }
-  for (int A = 0; A < 8; ++A)
-    for (const auto &st : stars) {
-      const int c = st[0];
-      const int t[4] = {8 * A + st[1], 8 * A + st[2], 8 * A + st[3], 8 * A + st[4]};
-      int others[7], n = 0;
-      for (int o = 0; o < 8; ++o)
-        if (o != A) others[n++] = o;
-      const int oct1[4] = {A, others[0], others[1], others[2]};
-      const int oct2[4] = {others[3], others[4], others[5], others[6]};
-      // inside A: {s, t, j} with j at or above the pair's larger index
-      auto valid = [&](int f, int j) {
-        return j / 8 != A || j % 8 >= std::max(c, st[1 + f]);
-      };
-      quarter(8 * A + c, t, oct1, valid);
-      quarter(8 * A + c, t, oct2, all);
-    }
-  // (3) degree 2 across octets: octet B < 7 takes j from B-1, B-2, B-3
-  // (mod 7) and from octet 7
-  for (int B = 0; B < 7; ++B) {
-    const int oct[4] = {(B + 6) % 7, (B + 5) % 7, (B + 4) % 7, 7};
-    for (int h = 0; h < 2; ++h) {
-      const int t[4] = {8 * B + 4 * h, 8 * B + 4 * h + 1, 8 * B + 4 * h + 2, 8 * B + 4 * h + 3};
-      quarter(ONES, t, oct, all);
-    }
-  }
-  // (4) the rest: j = c with third factors ONE (degree 1) and b <= c in the
-  // octet of c (degree 2), then the degree-0 row
-  for (int c = 0; c < 64; ++c) {
-    std::vector<int> th{ONES};
-    for (int b = c / 8 * 8; b <= c; ++b) th.push_back(b);
-    for (size_t i0 = 0; i0 < th.size(); i0 += kGroupRows) {
-      LaneGroup g;
-      g.j = c;
-      g.l = ONES;
-      for (int f = 0; f < kGroupRows; ++f) {
-        const bool ok = i0 + f < th.size();
-        g.third[f] = ok ? th[i0 + f] : ONES;
-        g.valid[f] = ok;
-      }
-      lg.push_back(g);
-    }
-  }
-  lg.push_back({ONES, ONES, {ONES, ONES, ONES, ONES}, {true, false, false, false}});
-}
-
 }  // namespace
 
 bool build_state_groups(int dK, const TileOrder &to, StateGroups *out) {
@@ -314,10 +178,6 @@ bool build_state_groups(int dK, const TileOrder &to, StateGroups *out) {
       if (g.third[f] == PAD) g.third[f] = ONES;
     lg.push_back(g);
   };
-  if (dK == 64) {
-    groups_uniform64(lg);
-    if (lg.empty()) return false;
-  } else {
   // degree 3, three distinct octets gi < gj < gl: third factor 8 gi + 4 ahi + f
   // (uniform in each warp), shared x_j x_l over the octets gj, gl
   for (int gi = 0; gi < G; ++gi)
@@ -361,7 +221,6 @@ bool build_state_groups(int dK, const TileOrder &to, StateGroups *out) {
   // degree 1 and degree 0
   for (int u0 = 0; u0 < dK; u0 += kGroupRows) add(ONES, ONES, u0, u0 + 1, u0 + 2, u0 + 3);
   add(ONES, ONES, ONES, PAD, PAD, PAD);
-  }
   while (lg.size() % 128) add(ONES, ONES, PAD, PAD, PAD, PAD);
 
   const int n_items = (int)(lg.size() / 128);

@@ -101,13 +101,14 @@ bool build_tile_order(int dK, TileOrder *out);
 // third (x_i0 .. x_i3), so per token it loads 2 + kGroupRows factor rows for
 // kGroupRows monomials instead of 3 per monomial.  A lane group is one such
 // set; an item is 128 lane groups (the 128 TMEM lanes) x kGroupRows rows (the
-// item's kGroupRows 128-row state tiles).  dK = 64: every warp (32 lanes, one
-// TMEM lane quarter) has one x_l and one x_i_f per row f for all its lanes
-// (broadcast loads) and its own factors x_j in four whole index octets (no
-// bank conflicts); the assignment of monomials to such quarter-units is
-// described in tile_order.cu.  dK = 32: degree 3 over three distinct octets
-// (shared x_j x_l, third factor uniform across each warp), degree 3 with a
-// pair inside one octet, degree 3 inside one octet, degree 2, 1, 0.  Unused
+// item's kGroupRows 128-row state tiles).  Groups, in order: degree 3 over
+// three distinct index octets (shared x_j x_l, third factor from the lowest
+// octet, uniform across each warp); degree 3 with a pair inside one octet
+// (shared pair, third factor from another octet, uniform across runs of 252
+// groups); degree 3 inside one octet; degree 2 (shared x_w and ones); degree
+// 1; degree 0.  (Groups whose second and third factors are one row for a
+// whole warp, with the own factors in whole octets, measured 5 % slower in the
+// state kernel at dK = 64 and are not used.)  Unused
 // rows of a group are padding (weight 0, no basis row); the tile order's
 // empty slots are given to padding rows, so that writing every row's slot
 // writes every snapshot column (zeros on the empty ones).

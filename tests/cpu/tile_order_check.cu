@@ -166,27 +166,6 @@ int check_groups(int dK) {
     }
   for (int64_t r = 0; r < hb.m; ++r) bad += row_hits[r] != 1;
   for (size_t k = 0; k < slot_hits.size(); ++k) bad += slot_hits[k] != 1;
-  // dK = 64: in almost every warp (32 lanes) the second and the third factors
-  // are one row for all lanes (broadcast loads) and the own factors of each
-  // 8-lane phase are 8 rows of distinct residues mod 8 (no bank conflict)
-  int uniform = 0, quarters = 0;
-  for (int it = 0; it < sg.n_items; ++it)
-    for (int q = 0; q < 4; ++q) {
-      bool ok = true;
-      const uint64_t i0 = sg.lane_idx[(size_t)it * 128 + 32 * q];
-      for (int lane = 0; lane < 32; ++lane) {
-        const uint64_t ix = sg.lane_idx[(size_t)it * 128 + 32 * q + lane];
-        if ((ix >> 8) != (i0 >> 8)) ok = false;
-        const uint64_t first = sg.lane_idx[(size_t)it * 128 + 32 * q + (lane & ~7)];
-        if ((ix & 7) != (uint64_t)(lane & 7) || ((ix & 0xff) >> 3) != ((first & 0xff) >> 3))
-          ok = false;
-      }
-      uniform += ok;
-      ++quarters;
-    }
-  printf("dK %d: %d state items, bad %ld, %d of %d warp quarters uniform\n", dK, sg.n_items, bad,
-         uniform, quarters);
-  if (dK == 64 && uniform < quarters - 8) ++bad;
   return bad ? 1 : 0;
 }
 
