@@ -46,6 +46,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <type_traits>
 
 #include "sata_internal.h"
 #include "tc_common.cuh"
@@ -406,76 +407,84 @@ __global__ void __launch_bounds__(kUThreads, 1)
 #pragma unroll
       for (int f = 0; f < kT; ++f)
         oi[f] = row_off((uint32_t)((ix >> (16 + 8 * ((un.f0 + f) & (kGroupRows - 1)))) & 0xff));
-      const int nr = un.nr;
-      for (int a = 0; ok && a < nA; ++a, ++ia) {
-        const int as = ia % kAS;
-        const uint32_t box = 2 * ia + hf;   // this warp's K/V box (global counter)
-        const uint32_t kv = box % kKS;
-        if (!(ok = mbar_wait(&kv_full[kv], (box / kKS) & 1, abort_flag, p.err, p.wait_limit)))
-          break;
-        if (ia >= kAS) {
-          if (!(ok = mbar_wait(&a_empty[as], ((ia / kAS) - 1) & 1, abort_flag, p.err,
-                               p.wait_limit)))
+      auto run_unit = [&](auto nr_c) {
+        constexpr int NR = decltype(nr_c)::value;  // tiles of this unit
+        for (int a = 0; ok && a < nA; ++a, ++ia) {
+          const int as = ia % kAS;
+          const uint32_t box = 2 * ia + hf;   // this warp's K/V box (global counter)
+          const uint32_t kv = box % kKS;
+          if (!(ok = mbar_wait(&kv_full[kv], (box / kKS) & 1, abort_flag, p.err, p.wait_limit)))
             break;
-          // the MMAs of A stage ia - kAS are complete: its box of this half
-          // can be reloaded
+          if (ia >= kAS) {
+            if (!(ok = mbar_wait(&a_empty[as], ((ia / kAS) - 1) & 1, abort_flag, p.err,
+                                 p.wait_limit)))
+              break;
+            // the MMAs of A stage ia - kAS are complete: its box of this half
+            // can be reloaded
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&kv_empty[(2 * (ia - kAS) + hf) % kKS]);
+          }
+          const uint32_t kt = smem_u32(sKT) + kv * S::UKTh;
+          const uint32_t aj = kt + oj, al = kt + ol;
+          uint32_t ai[kT];
+  #pragma unroll
+          for (int f = 0; f < kT; ++f) ai[f] = kt + oi[f];
+          const uint32_t tcol = tmem + tl + S::UColA + as * kT * (kAT / 2) + 32 * hf;
+          // 8 tokens per 16-byte chunk of a K^T row; the loads of chunk c + 1
+          // are issued before the products of chunk c, and each half of the 64
+          // tokens goes to TMEM as soon as it is complete
+          uint4 xj = lds128(aj), xl = lds128(al), xi[kT];
+  #pragma unroll
+          for (int f = 0; f < kT; ++f)
+            if (f < NR) xi[f] = lds128(ai[f]);
+          uint32_t out[kT][32];
+  #pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 nj, nl, ni[kT];
+            if (c < 7) {
+              const uint32_t sw = (uint32_t)(c + 1) << 4;
+              nj = lds128(aj ^ sw);
+              nl = lds128(al ^ sw);
+  #pragma unroll
+              for (int f = 0; f < kT; ++f)
+                if (f < NR) ni[f] = lds128(ai[f] ^ sw);
+            }
+            const uint4 pr = make_uint4(bmul2(xj.x, xl.x), bmul2(xj.y, xl.y), bmul2(xj.z, xl.z),
+                                        bmul2(xj.w, xl.w));
+  #pragma unroll
+            for (int f = 0; f < kT; ++f) {
+              if (f >= NR) continue;
+              out[f][4 * c + 0] = bmul2(xi[f].x, pr.x);
+              out[f][4 * c + 1] = bmul2(xi[f].y, pr.y);
+              out[f][4 * c + 2] = bmul2(xi[f].z, pr.z);
+              out[f][4 * c + 3] = bmul2(xi[f].w, pr.w);
+            }
+            if (c == 3 || c == 7) {
+  #pragma unroll
+              for (int f = 0; f < kT; ++f)
+                if (f < NR)
+                  tmem_st16(tcol + f * (kAT / 2) + (c == 3 ? 0 : 16),
+                            *reinterpret_cast<const uint32_t(*)[16]>(&out[f][c == 3 ? 0 : 16]));
+            }
+            if (c < 7) {
+              xj = nj;
+              xl = nl;
+  #pragma unroll
+              for (int f = 0; f < kT; ++f) xi[f] = ni[f];
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&kv_empty[(2 * (ia - kAS) + hf) % kKS]);
+          if (lane == 0) mbar_arrive(&a_full[as]);
         }
-        const uint32_t kt = smem_u32(sKT) + kv * S::UKTh;
-        const uint32_t aj = kt + oj, al = kt + ol;
-        uint32_t ai[kT];
-#pragma unroll
-        for (int f = 0; f < kT; ++f) ai[f] = kt + oi[f];
-        const uint32_t tcol = tmem + tl + S::UColA + as * kT * (kAT / 2) + 32 * hf;
-        // 8 tokens per 16-byte chunk of a K^T row; the loads of chunk c + 1
-        // are issued before the products of chunk c, and each half of the 64
-        // tokens goes to TMEM as soon as it is complete
-        uint4 xj = lds128(aj), xl = lds128(al), xi[kT];
-#pragma unroll
-        for (int f = 0; f < kT; ++f)
-          if (f < nr) xi[f] = lds128(ai[f]);
-        uint32_t out[kT][32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 nj, nl, ni[kT];
-          if (c < 7) {
-            const uint32_t sw = (uint32_t)(c + 1) << 4;
-            nj = lds128(aj ^ sw);
-            nl = lds128(al ^ sw);
-#pragma unroll
-            for (int f = 0; f < kT; ++f)
-              if (f < nr) ni[f] = lds128(ai[f] ^ sw);
-          }
-          const uint4 pr = make_uint4(bmul2(xj.x, xl.x), bmul2(xj.y, xl.y), bmul2(xj.z, xl.z),
-                                      bmul2(xj.w, xl.w));
-#pragma unroll
-          for (int f = 0; f < kT; ++f) {
-            if (f >= nr) continue;
-            out[f][4 * c + 0] = bmul2(xi[f].x, pr.x);
-            out[f][4 * c + 1] = bmul2(xi[f].y, pr.y);
-            out[f][4 * c + 2] = bmul2(xi[f].z, pr.z);
-            out[f][4 * c + 3] = bmul2(xi[f].w, pr.w);
-          }
-          if (c == 3 || c == 7) {
-#pragma unroll
-            for (int f = 0; f < kT; ++f)
-              if (f < nr)
-                tmem_st16(tcol + f * (kAT / 2) + (c == 3 ? 0 : 16),
-                          *reinterpret_cast<const uint32_t(*)[16]>(&out[f][c == 3 ? 0 : 16]));
-          }
-          if (c < 7) {
-            xj = nj;
-            xl = nl;
-#pragma unroll
-            for (int f = 0; f < kT; ++f) xi[f] = ni[f];
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[as]);
-      }
+      };
+      // the unit's tile count as a constant: a loop body that tests it per
+      // tile runs markedly slower
+      if (un.nr == kT)
+        run_unit(std::integral_constant<int, kT>{});
+      else
+        run_unit(std::integral_constant<int, 1>{});
     }
   }
 
@@ -907,26 +916,60 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint8_t *qrow = sQ + b * kRTile + row * kRow;
     const uint32_t tl = (uint32_t)(32 * (gw & 3)) << 16;
     const int n_stages = (p.n_tiles + kRTS - 1) / kRTS;
-    for (int i = 0; ok && i < n_stages; ++i) {
-      const int st = i % kRStages;
-      if (i >= kRStages && !(ok = mbar_wait(&a_empty[st], ((i / kRStages) - 1) & 1, abort_flag,
-                                            p.err, p.wait_limit)))
-        break;
-      // this thread's token is TMEM lane `row` of block b; a tile's 64
-      // features are 32 packed columns
-      const uint32_t acol = tmem + tl + ColA + (st * 2 + b) * kRTS * 32;
+    const uint32_t rsw = (uint32_t)(row & 7);
+    static_assert(kRTS == 2, "stages of two tiles");
+    // One loop per run of the tile order (tile_order.h): the OUTER tiles of
+    // three distinct octets in pairs (C(G,3) x 8 tiles), then the BC tiles
+    // variant by variant (G (G-1) / 2 tiles each), then the rest tile by tile.
+    // A loop whose body holds one generation path runs about twice as fast as
+    // one that dispatches among all of them.
+    int i = 0;
+    auto run = [&](int i_end, auto gen) {
+      for (; ok && i < i_end; ++i) {
+        const int st = i % kRStages;
+        if (i >= kRStages && !(ok = mbar_wait(&a_empty[st], ((i / kRStages) - 1) & 1,
+                                              abort_flag, p.err, p.wait_limit)))
+          break;
+        // this thread's token is TMEM lane `row` of block b; a tile's 64
+        // features are 32 packed columns
+        gen(i, tmem + tl + ColA + (st * 2 + b) * kRTS * 32);
+        tmem_st_wait();
+        if (!(ok = mbar_wait(&b_full[i % kRBS], (i / kRBS) & 1, abort_flag, p.err, p.wait_limit)))
+          break;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[st]);
+      }
+    };
+    constexpr int kOuterStages = S::G * (S::G - 1) * (S::G - 2) / 6 * 4;
+    constexpr int kBcStages = S::G * (S::G - 1) / 4;
+    run(std::min(kOuterStages, n_stages), [&](int i, uint32_t acol) {
+      uint32_t out0[32], out1[32];
+      gen_outer_pair(sTiles[2 * i], qrow, rsw, p.W, out0, out1);
+      tmem_st32(acol, out0);
+      tmem_st32(acol + 32, out1);
+    });
+    auto bc = [&](auto t_c) {
+      return [&, t_c](int i, uint32_t acol) {
+        gen_store_bc2<S::G, decltype(t_c)::value>(sTiles[2 * i], sTiles[2 * i + 1], qrow, rsw,
+                                                  p.W, acol);
+      };
+    };
+    run(std::min(kOuterStages + 1 * kBcStages, n_stages), bc(std::integral_constant<int, 0>{}));
+    run(std::min(kOuterStages + 2 * kBcStages, n_stages), bc(std::integral_constant<int, 1>{}));
+    run(std::min(kOuterStages + 3 * kBcStages, n_stages), bc(std::integral_constant<int, 2>{}));
+    run(std::min(kOuterStages + 4 * kBcStages, n_stages), bc(std::integral_constant<int, 3>{}));
+    run(std::min(kOuterStages + 5 * kBcStages, n_stages), bc(std::integral_constant<int, 4>{}));
+    run(std::min(kOuterStages + 6 * kBcStages, n_stages), bc(std::integral_constant<int, 5>{}));
+    run(std::min(kOuterStages + 7 * kBcStages, n_stages), bc(std::integral_constant<int, 6>{}));
+    run(std::min(kOuterStages + 8 * kBcStages, n_stages), bc(std::integral_constant<int, 7>{}));
+    run(std::min(kOuterStages + 9 * kBcStages, n_stages), bc(std::integral_constant<int, 8>{}));
+    run(n_stages, [&](int i, uint32_t acol) {
       const TileDesc pad{T_PAD, 0, 0, 0, 0, 0, 0, 0};
       const TileDesc d0 = kRTS * i < p.n_tiles ? sTiles[kRTS * i] : pad;
       const TileDesc d1 = kRTS * i + 1 < p.n_tiles ? sTiles[kRTS * i + 1] : pad;
-      static_assert(kRTS == 2, "stages of two tiles");
-      gen_store_stage<S::G>(d0, d1, qrow, (uint32_t)(row & 7), p.W, acol);
-      tmem_st_wait();
-      if (!(ok = mbar_wait(&b_full[i % kRBS], (i / kRBS) & 1, abort_flag, p.err, p.wait_limit)))
-        break;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[st]);
-    }
+      gen_store_stage<S::G>(d0, d1, qrow, rsw, p.W, acol);
+    });
   }
 
   tc_fence_before();

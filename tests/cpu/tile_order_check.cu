@@ -96,6 +96,16 @@ int check(int dK, int want_tiles, bool unit_weights) {
       }
     }
   }
+  // the runs the readout's generator loops assume: C(G,3) x 8 OUTER tiles in
+  // pairs for the two-tile path, then G (G-1) / 2 BC tiles of each variant
+  {
+    const int n3 = G * (G - 1) * (G - 2) / 6 * 8, nbc = G * (G - 1) / 2;
+    for (int t = 0; t < n3; t += 2)
+      if (!tc::outer_pair_ok(to.tiles[t], to.tiles[t + 1])) ++bad;
+    for (int v = 0; v < 9; ++v)
+      for (int t = n3 + v * nbc; t < n3 + (v + 1) * nbc; ++t)
+        if (to.tiles[t].type != T_BC || to.tiles[t].variant != v) ++bad;
+  }
   // the readout's two-tile path equals the one-tile path bit for bit
   long pair_bad = 0, pairs = 0;
   for (int trial = 0; trial < 4; ++trial) {
