@@ -523,6 +523,7 @@ def run_ours(args, rank, world, local_rank):
     decode["mixed_state"] = time_decode(
         mixed_step, m_lo * (dw["dV"] + 1) * 4 + (dm - m_lo) * (dw["dV"] + 1) * 2,
         f"rows of degree <= 2 fp32 ({m_lo}/head), degree 3 fp16 ({dm - m_lo}/head)")
+    variants = time_variants(sata, stream, dev, flush, pk, rank)
     clocks = sampler.stop()
     assert sata.sata_get_error() == sata.SATA_OK
 
@@ -536,13 +537,78 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "prefill: 256 MiB L2 flush between timed steps; decode: 3.19 GB fp32 "
                          "(1.66 GB mixed) state > L2",
                    "decode_steps": nsteps},
-        "roofline": roof, "decode": decode, "prefill_dk32": prefill_dk32, "e2e": e2e,
+        "roofline": roof, "decode": decode, "prefill_dk32": prefill_dk32, "variants": variants,
+        "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     return line
+
+
+# --------------------------------------------------------------- variants
+def time_variants(sata, stream, dev, flush, pk, rank, steps=5, warmup=3):
+    """Short measurements of the variants beyond the two benchmark workloads:
+    P = 5 decode at d_K = 64 (its state is 212 MB per head) and two prefills
+    on the CUDA-core path (many small fp32 heads; P = 5 bf16)."""
+    import torch
+    from sata_inputs import make_qkv
+
+    def timed(fn, flush_l2):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(steps):
+            if flush_l2:
+                flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    out = {}
+    # decode, P = 5, d_K = d_V = 64, B = 1, H = 2, state of a 64-token prefill
+    B, H, N, d, P = 1, 2, 64, 64, 5
+    m = basis_m(d, P)
+    q, k, v = (t.to(dev) for t in make_qkv(B, H, N + 1, d, d, seed=20261210 + 1000 * rank,
+                                            dtype="bf16"))
+    st = torch.empty(B, H, m, d + 1, device=dev)
+    sata.sata_prefill(q[:, :, :N].contiguous(), k[:, :, :N].contiguous(), v[:, :, :N].contiguous(),
+                      torch.empty(B, H, N, d, device=dev), st, B, H, N, d, d, P, torch.bfloat16,
+                      stream)
+    qt, kt, vt = (x[:, :, N].contiguous() for x in (q, k, v))
+    o = torch.empty(B, H, d, device=dev)
+    ms = timed(lambda: sata.sata_decode_step(qt, kt, vt, st, o, B, H, d, d, P, torch.bfloat16,
+                                             stream), False)
+    nbytes = 2 * B * H * m * (d + 1) * 4
+    out["decode_p5_dk64"] = {
+        "workload": "decode B=1,H=2,dK=dV=64,P=5 fp32 state (814385 rows/head, 212 MB/head)",
+        "ms_per_step": ms, "tokens_per_s": B / (ms / 1e3),
+        "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "unit": "GB/s",
+                     "peak": pk["hbm_gbs"], "frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                     "algorithmic_bytes_per_launch": nbytes}}
+    del q, k, v, st
+    # prefill on the CUDA-core path: many small fp32 heads, and P = 5 bf16
+    for key, (B, H, N, d, P, dt, tdt) in {
+            "prefill_f32_dk16_h64": (4, 64, 1024, 16, 4, "f32", torch.float32),
+            "prefill_bf16_dk16_p5": (1, 8, 4096, 16, 5, "bf16", torch.bfloat16)}.items():
+        m = basis_m(d, P)
+        q, k, v = (t.to(dev) for t in make_qkv(B, H, N, d, d, seed=20261211 + 1000 * rank,
+                                                dtype=dt))
+        o = torch.empty(B, H, N, d, device=dev)
+        st = torch.empty(B, H, m, d + 1, device=dev)
+        ms = timed(lambda: sata.sata_prefill(q, k, v, o, st, B, H, N, d, d, P, tdt, stream), True)
+        out[key] = {"workload": f"prefill B={B},H={H},N={N},dK=dV={d},P={P} {dt} (CUDA cores)",
+                    "ms_per_step": ms, "tokens_per_s": B * N / (ms / 1e3),
+                    "head_tokens_per_s": B * H * N / (ms / 1e3)}
+        del q, k, v, o, st
+    torch.cuda.synchronize()
+    return out
 
 
 # --------------------------------------------------------------- reference arm
