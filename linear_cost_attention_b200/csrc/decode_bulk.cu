@@ -215,29 +215,61 @@ __global__ void __launch_bounds__((D1 * BulkShape<D1>::KB + 31) / 32 * 32 + 32)
       ok = mbar_wait(&full[st], (i / kStages) & 1, &abort_flag, p.err, p.wait_limit);
       if (!ok) continue;  // the next barrier stops every compute thread
       if (worker) {
+        // a segment inside one head (all but a few) takes the loops without
+        // a per-row head check; y takes the updated value before it is
+        // rounded to the stored precision
+        const int rows = hi ? kRows16 : kRows32;
+        const int h0 = __float_as_int(meta[slot][0].z);
+        const bool one_head = h0 == __float_as_int(meta[slot][rows - 1].z);
+        if (one_head) use_head(h0);
+        const float2 *mq = reinterpret_cast<const float2 *>(meta[slot]);  // (phi_q, phi_k) per row
         if (hi) {
           __half *sg = reinterpret_cast<__half *>(ring + st * SB);
+          if (one_head) {
+#pragma unroll 8
+            for (int j = 0; j < kRows16 / KB; ++j) {
+              const int rl = ro + KB * j;
+              const float2 mt = mq[2 * rl];
+              const int e = rl * D1 + c;
+              const float sn = fmaf(mt.y, vc, __half2float(sg[e]));
+              sg[e] = __float2half_rn(sn);
+              acc = fmaf(mt.x, sn, acc);
+            }
+          } else {
 #pragma unroll 4
-          for (int j = 0; j < kRows16 / KB; ++j) {
-            const int rl = ro + KB * j;
-            const float4 mt = meta[slot][rl];
-            use_head(__float_as_int(mt.z));
-            const int e = rl * D1 + c;
-            const __half hn = __float2half_rn(fmaf(mt.y, vc, __half2float(sg[e])));
-            sg[e] = hn;
-            acc = fmaf(mt.x, __half2float(hn), acc);
+            for (int j = 0; j < kRows16 / KB; ++j) {
+              const int rl = ro + KB * j;
+              const float4 mt = meta[slot][rl];
+              use_head(__float_as_int(mt.z));
+              const int e = rl * D1 + c;
+              const float sn = fmaf(mt.y, vc, __half2float(sg[e]));
+              sg[e] = __float2half_rn(sn);
+              acc = fmaf(mt.x, sn, acc);
+            }
           }
         } else {
           float *sg = reinterpret_cast<float *>(ring + st * SB);
+          if (one_head) {
+#pragma unroll 8
+            for (int j = 0; j < kRows32 / KB; ++j) {
+              const int rl = ro + KB * j;
+              const float2 mt = mq[2 * rl];
+              const int e = rl * D1 + c;
+              const float sn = fmaf(mt.y, vc, sg[e]);
+              sg[e] = sn;
+              acc = fmaf(mt.x, sn, acc);
+            }
+          } else {
 #pragma unroll 4
-          for (int j = 0; j < kRows32 / KB; ++j) {
-            const int rl = ro + KB * j;
-            const float4 mt = meta[slot][rl];
-            use_head(__float_as_int(mt.z));
-            const int e = rl * D1 + c;
-            const float sn = fmaf(mt.y, vc, sg[e]);
-            sg[e] = sn;
-            acc = fmaf(mt.x, sn, acc);
+            for (int j = 0; j < kRows32 / KB; ++j) {
+              const int rl = ro + KB * j;
+              const float4 mt = meta[slot][rl];
+              use_head(__float_as_int(mt.z));
+              const int e = rl * D1 + c;
+              const float sn = fmaf(mt.y, vc, sg[e]);
+              sg[e] = sn;
+              acc = fmaf(mt.x, sn, acc);
+            }
           }
         }
       }
