@@ -259,6 +259,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
           if (!(ok = mbar_wait(d_ready, units & 1, abort_flag, p.err, p.wait_limit))) break;
           tc_fence_after();
         }
+        // the unit's next event (chunk boundary or last stage), kept as a
+        // counter: this thread's instructions between MMAs are its cost
+        int next_event = std::min(a_per_chunk, nA) - 1;
         for (int a = 0; ok && a < nA; ++a, ++ia) {
           const int as = ia % kAS;
           // a_full also covers kv_full: every generator warp waited on its K/V
@@ -290,7 +293,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
                           k > 0 ? 1u : acc0);
           }
           mma_commit(&a_empty[as]);
-          if (is_event(a)) {
+          if (a == next_event) {
+            next_event = std::min(next_event + a_per_chunk, nA - 1);
             mma_commit(&snap_full[f]);
             ++events;
             after_event = true;
