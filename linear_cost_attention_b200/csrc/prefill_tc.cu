@@ -820,8 +820,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       if (ok) intra(false);
       if (ok && inter) {
-        const uint32_t b0 = smem_u32(sB);
-        const int n_stages = (p.n_tiles + kRTS - 1) / kRTS;
+        // the tile count is even (the host pads it), so every stage holds
+        // kRTS = 2 tiles; descriptors step from one base (a snapshot tile is
+        // RB bytes, RB >> 4 in the address field; a K-step 32 bytes, 2)
+        const uint64_t bd_base = smem_desc_sw128(smem_u32(sB), 16, 1024);
+        const int n_stages = p.n_tiles / kRTS;
         for (int i = 0; i < n_stages; ++i) {
           const int st = i % kRStages, bs = i % kRBS;
           // a_full also covers b_full: the generator warps wait on the snapshot
@@ -829,9 +832,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(&a_full[st], (i / kRStages) & 1, abort_flag, p.err, p.wait_limit)))
             break;
           tc_fence_after();
-          const int nt = min(kRTS, p.n_tiles - kRTS * i);
-          for (int t = 0; t < nt; ++t) {
-            const uint64_t bd = smem_desc_sw128(b0 + (bs * kRTS + t) * S::RB, 16, 1024);
+#pragma unroll
+          for (int t = 0; t < kRTS; ++t) {
+            const uint64_t bd = bd_base + (uint64_t)((bs * kRTS + t) * (S::RB >> 4));
             const uint32_t ad = tmem + ColA + ((st * 2 + b) * kRTS + t) * 32;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
